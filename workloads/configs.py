@@ -1,0 +1,97 @@
+"""The five synthetic single-layer workloads and small variants of them.
+
+Shapes follow the Qwen2.5-1M report explainer (0h-n0.github.io, "Inference
+framework" / "Chunked Prefill": 32,768-token chunks, last 64 queries of each
+chunk drive selection; Table 2: final RoPE base 10,000,000) and the two model
+shapes: Qwen2.5-7B (28 query / 4 KV heads, head_dim 128) and a 14B-shaped layer
+(40 / 8). DCA constants: chunk size C as given per workload, local window
+W = C / 32, stride S = C - W (the reading recorded in the design doc).
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, replace
+from typing import Optional
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    hq: int
+    hkv: int
+    seq_len: int
+    seed: int
+    n_planted: int
+    kv_budget: int  # base vertical budget k_v
+    ks_budget: int  # base slash budget k_s
+    refine_tau: Optional[float]  # None: no refinement
+    dca_chunk: Optional[int] = None  # DCA chunk size C (None: continuous RoPE)
+    chunk: int = 32768  # prefill chunk length
+    head_dim: int = 128
+    rope_base: float = 1.0e7
+    last_q: int = 64
+
+    @property
+    def dca_window(self) -> Optional[int]:
+        return None if self.dca_chunk is None else self.dca_chunk // 32
+
+    @property
+    def dca_stride(self) -> Optional[int]:
+        return None if self.dca_chunk is None else self.dca_chunk - self.dca_chunk // 32
+
+    @property
+    def group(self) -> int:
+        return self.hq // self.hkv
+
+    @property
+    def n_chunks(self) -> int:
+        return (self.seq_len + self.chunk - 1) // self.chunk
+
+    def chunk_bounds(self, c: int) -> tuple[int, int]:
+        cs = c * self.chunk
+        return cs, min(cs + self.chunk, self.seq_len)
+
+
+WORKLOADS: dict[int, Workload] = {
+    1: Workload("cfg1_h2x1_n4k", hq=2, hkv=1, seq_len=4096, seed=0, n_planted=16,
+                kv_budget=256, ks_budget=256, refine_tau=None),
+    2: Workload("cfg2_qwen7b_n32k_refine", hq=28, hkv=4, seq_len=32768, seed=1, n_planted=64,
+                kv_budget=1000, ks_budget=2048, refine_tau=0.9),
+    3: Workload("cfg3_qwen7b_n128k_4chunks_refine", hq=28, hkv=4, seq_len=131072, seed=2,
+                n_planted=64, kv_budget=1000, ks_budget=2048, refine_tau=0.9),
+    4: Workload("cfg4_14b_n256k_dca64k", hq=40, hkv=8, seq_len=262144, seed=3, n_planted=256,
+                kv_budget=1000, ks_budget=2048, refine_tau=None, dca_chunk=65536),
+    5: Workload("cfg5_14b_n1m_dca256k_refine", hq=40, hkv=8, seq_len=1048576, seed=4,
+                n_planted=1024, kv_budget=1000, ks_budget=2048, refine_tau=0.9,
+                dca_chunk=262144),
+}
+
+
+def small_workload(base: int, seq_len: int, chunk: int, *, hq: Optional[int] = None,
+                   hkv: Optional[int] = None, n_planted: Optional[int] = None,
+                   kv_budget: Optional[int] = None, ks_budget: Optional[int] = None,
+                   dca_chunk: Optional[int] = None, seed: Optional[int] = None,
+                   refine_tau: Optional[float] = -1.0, head_dim: Optional[int] = None,
+                   name: Optional[str] = None) -> Workload:
+    """A reduced copy of workload `base` (same generator recipe, smaller sizes)."""
+    w = WORKLOADS[base]
+    kw = dict(seq_len=seq_len, chunk=chunk)
+    if hq is not None:
+        kw["hq"] = hq
+    if hkv is not None:
+        kw["hkv"] = hkv
+    if n_planted is not None:
+        kw["n_planted"] = n_planted
+    if kv_budget is not None:
+        kw["kv_budget"] = kv_budget
+    if ks_budget is not None:
+        kw["ks_budget"] = ks_budget
+    if dca_chunk is not None:
+        kw["dca_chunk"] = dca_chunk
+    if seed is not None:
+        kw["seed"] = seed
+    if refine_tau != -1.0:
+        kw["refine_tau"] = refine_tau
+    if head_dim is not None:
+        kw["head_dim"] = head_dim
+    kw["name"] = name or f"{w.name}_small_n{seq_len}_c{chunk}"
+    return replace(w, **kw)
