@@ -1,0 +1,471 @@
+#!/usr/bin/env python3
+"""Benchmark of the sparse chunked-prefill hot path of one attention layer.
+
+One step = the whole path for one layer over the synthetic workload: for every
+32K-query chunk, estimation (last 64 queries against the growing KV), top-k
+vertical/slash selection with refinement by attention recall where the workload
+has a threshold, and the sparse attention of the chunk's rows (with DCA
+positions where the workload uses DCA). Inputs are resident in HBM when the
+timed region starts; L2 is flushed between steps. The `e2e` figure repeats the
+step through the same public API from pinned host buffers, host<->device copies
+of the inputs and of the output inside the timed region.
+
+Multi-GPU (torchrun): every rank prefills its own independent layer (seed
+offset by rank), no collective on the data path; value = all tokens / max rank
+time ("weak" scaling).
+
+--impl reference: the CPU oracle (oracle/) timed on a bounded sample of the same
+workload, extrapolated to the layer.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+from dataclasses import replace
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from workloads import WORKLOADS, generate_head, structure  # noqa: E402
+
+METRIC = "sparse-prefill tokens/s per layer; executed TFLOP/s and % of B200 BF16 peak"
+FLOP_PER_TILE = 4 * 128 * 128 * 128  # QK^T and PV of one executed 128-query x 128-key tile
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def parse():
+    p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=5)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--config", type=int, default=2, choices=sorted(WORKLOADS))
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--max-iters", type=int, default=19)
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons with nvidia-smi during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            bus = torch.cuda.get_device_properties(self.idx).pci_bus_id
+            sel = ["--id=" + bus] if bus else ["-i", str(self.idx)]
+        except Exception:
+            sel = ["-i", str(self.idx)]
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", *sel, "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- the GPU path
+class Layer:
+    """One layer's inputs on the device, the library context and per-chunk buffers."""
+
+    def __init__(self, w, device, max_iters):
+        import sparse_attention_estimate_b200 as vsb
+
+        self.vsb = vsb
+        self.w = w
+        self.dev = device
+        self.max_iters = max_iters
+        st = structure(w)
+        t0 = time.time()
+        self.q = torch.empty(w.hq, w.seq_len, 128, dtype=torch.bfloat16, device=device)
+        self.k = torch.empty(w.hkv, w.seq_len, 128, dtype=torch.bfloat16, device=device)
+        self.v = torch.empty(w.hkv, w.seq_len, 128, dtype=torch.bfloat16, device=device)
+        for name, t, nh in (("q", self.q, w.hq), ("k", self.k, w.hkv), ("v", self.v, w.hkv)):
+            for h in range(nh):
+                t[h].copy_(generate_head(w, name, h, st=st))
+        log(f"[bench] generated {w.name} in {time.time() - t0:.1f}s")
+        self.out = torch.empty_like(self.q)
+        self.lse = torch.empty(w.hq, w.seq_len, dtype=torch.float32, device=device)
+        C = w.dca_chunk
+        cfg = vsb.Config(hq=w.hq, hkv=w.hkv, rope_base=w.rope_base, last_q=w.last_q, dca_chunk=C,
+                         dca_window=w.dca_window if C else None)
+        self.ctx = vsb.Context(cfg, max_seq=w.seq_len, max_chunk=min(w.chunk, w.seq_len), device=device)
+        e_max = w.seq_len
+        self.vert = torch.empty(w.hq, e_max, dtype=torch.float32, device=device)
+        self.slash = torch.empty_like(self.vert)
+        self.lse_est = torch.empty(w.hq, 64, dtype=torch.float32, device=device)
+        self.base_v = torch.full((w.hq,), w.kv_budget, dtype=torch.int32, device=device)
+        self.base_s = torch.full((w.hq,), w.ks_budget, dtype=torch.int32, device=device)
+        self.kv = torch.empty_like(self.base_v)
+        self.ks = torch.empty_like(self.base_s)
+        self.recall = torch.empty(w.hq, dtype=torch.float32, device=device)
+        self.sets = (torch.empty(w.hq, e_max, dtype=torch.int32, device=device),
+                     torch.empty(w.hq, dtype=torch.int32, device=device),
+                     torch.empty(w.hq, e_max, dtype=torch.int32, device=device),
+                     torch.empty(w.hq, dtype=torch.int32, device=device))
+        self.chunks = [w.chunk_bounds(c) for c in range(w.n_chunks)]
+
+    def step(self, attn_events=None, stats=None, q=None, k=None, v=None):
+        """One pass of the whole hot path. attn_events: list of (start, stop) per
+        chunk, recorded around the attention kernel; stats: list receiving the
+        (executed tiles, useful pairs) of each chunk (synchronises)."""
+        w, ctx = self.w, self.ctx
+        q = self.q if q is None else q
+        k = self.k if k is None else k
+        v = self.v if v is None else v
+        ctx.reset()  # every step rotates its keys again
+        for ci, (cs, e) in enumerate(self.chunks):
+            vert, slash = self.vert[:, :e], self.slash[:, :e]
+            ctx.estimate(q, cs, k, e, out=(self.vert, self.slash, self.lse_est), full=True)
+            self.kv.copy_(self.base_v)
+            self.ks.copy_(self.base_s)
+            if w.refine_tau is None:
+                ctx.select(self.vert, self.slash, e, self.kv, self.ks, sets=self.sets)
+            else:
+                ctx.refine(q, cs, k, e, self.vert, self.slash, self.lse_est, w.refine_tau, self.kv, self.ks,
+                           max_iters=self.max_iters, sets=self.sets, recall=self.recall, full=True)
+            if attn_events is not None:
+                ctx.set_prefill_events(*attn_events[ci])
+            ctx.sparse_prefill(q, cs, e, k, v, self.sets, out=self.out, lse=self.lse, full=True)
+            if attn_events is not None:
+                ctx.set_prefill_events(None, None)
+            if stats is not None:
+                stats.append(ctx.prefill_stats())
+            del vert, slash
+
+
+def flush_l2(buf):
+    buf.zero_()
+
+
+def run_ours(args, rank, world, device):
+    import sparse_attention_estimate_b200 as vsb
+    from sparse_attention_estimate_b200 import build as vsbuild
+
+    vsbuild.build()
+    vsb.load_library()
+    w = WORKLOADS[args.config]
+    if rank > 0:
+        w = replace(w, seed=w.seed + 1000 * rank)
+    lay = Layer(w, device, args.max_iters)
+    l2 = torch.empty(256 << 20, dtype=torch.uint8, device=device)  # > 126 MB L2
+    nchunks = len(lay.chunks)
+
+    def new_events():
+        evs = []
+        for _ in range(nchunks):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            b.record()
+            evs.append((a, b))
+        return evs
+
+    for _ in range(args.warmup):
+        flush_l2(l2)
+        lay.step()
+    torch.cuda.synchronize()
+    assert lay.ctx.status() == vsb.VS_OK, "device error during warm-up"
+    # executed tiles / useful pairs of one step (untimed; reads counters per chunk)
+    stats = []
+    lay.step(stats=stats)
+    executed = sum(s[0] for s in stats)
+    useful = sum(s[1] for s in stats)
+    # ---------------------------------------------------------------- timed region
+    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+    attn_ev = [new_events() for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    n0 = vsb.kernel_launches()
+    with ClockSampler(device.index or 0) as clk:
+        for i in range(args.steps):
+            flush_l2(l2)
+            step_ev[i][0].record()
+            lay.step(attn_events=attn_ev[i])
+            step_ev[i][1].record()
+        torch.cuda.synchronize()
+    launches = vsb.kernel_launches() - n0
+    if world > 1:
+        torch.distributed.barrier()
+    assert lay.ctx.status() == vsb.VS_OK, "device error in the timed region"
+    step_ms = [a.elapsed_time(b) for a, b in step_ev]
+    attn_ms = [sum(a.elapsed_time(b) for a, b in evs) for evs in attn_ev]
+    tot_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([tot_ms], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        tot_ms = float(t.item())
+    ms_per_step = tot_ms / args.steps
+    tokens = w.seq_len * args.steps * world
+    value = tokens / (tot_ms / 1e3)
+    attn_ms_step = sum(attn_ms) / args.steps
+    exec_flops = executed * FLOP_PER_TILE
+    useful_flops = useful * 4 * 128
+    pk, pk_src = peaks()
+    long_step = ms_per_step > 1000.0
+    peak = pk["bf16_tflops_sustained"] if long_step else pk["bf16_tflops"]
+    attn_tflops = exec_flops / (attn_ms_step / 1e3) / 1e12
+    res = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded generator: N(0,1) Q/K/V, planted verticals, 64-aligned band)",
+        "config": {
+            "workload": w.name, "seq_len": w.seq_len, "hq": w.hq, "hkv": w.hkv, "head_dim": 128,
+            "chunk": w.chunk, "n_chunks": nchunks, "dca": [w.dca_chunk, w.dca_window] if w.dca_chunk else None,
+            "budgets": [w.kv_budget, w.ks_budget], "refine_tau": w.refine_tau,
+            "parallelism": f"independent layer per GPU x{world}" if world > 1 else "single GPU",
+            "l2": "flushed between steps (256 MiB write)",
+        },
+        "executed_tflops": round(exec_flops / (ms_per_step / 1e3) / 1e12, 2),
+        "attn_executed_tflops": round(attn_tflops, 2),
+        "pct_bf16_peak": round(100 * attn_tflops / peak, 2),
+        "pct_bf16_peak_of": f"{pk_src} {'sustained' if long_step else 'burst'} {peak} TFLOP/s",
+        "useful_tflops": round(useful_flops / (ms_per_step / 1e3) / 1e12, 2),
+        "density_useful_over_executed": round(useful_flops / exec_flops, 4) if exec_flops else None,
+        "attn_ms_per_step": round(attn_ms_step, 3),
+        "roofline": {
+            "bound": "tensor", "kernel": "attn_kernel",
+            "achieved": round(attn_tflops, 2), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(attn_tflops / peak, 4), "traffic": None,
+            "peak_kind": f"{pk_src} {'sustained' if long_step else 'burst'} bf16",
+            "flop_per_launch": round(exec_flops / nchunks),
+        },
+        "gpu_launches": int(launches),
+        "clocks": clk.summary(),
+    }
+    # ---------------------------------------------------------------- end to end (host buffers)
+    if not args.no_e2e:
+        res["e2e"] = run_e2e(args, lay, l2, world, device)
+    return res, w, lay
+
+
+def run_e2e(args, lay, l2, world, device):
+    """Same step through the public API from pinned host memory: H2D of q, k, v
+    and D2H of the output inside the timed region."""
+    hq_h = lay.q.cpu().pin_memory()
+    hk_h = lay.k.cpu().pin_memory()
+    hv_h = lay.v.cpu().pin_memory()
+    out_h = torch.empty(lay.out.shape, dtype=lay.out.dtype).pin_memory()
+    dq, dk, dv = torch.empty_like(lay.q), torch.empty_like(lay.k), torch.empty_like(lay.v)
+
+    def e2e_step():
+        dq.copy_(hq_h, non_blocking=True)
+        dk.copy_(hk_h, non_blocking=True)
+        dv.copy_(hv_h, non_blocking=True)
+        lay.step(q=dq, k=dk, v=dv)
+        out_h.copy_(lay.out, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    for i in range(args.steps):
+        flush_l2(l2)
+        evs[i][0].record()
+        e2e_step()
+        evs[i][1].record()
+    torch.cuda.synchronize()
+    tot = sum(a.elapsed_time(b) for a, b in evs)
+    if world > 1:
+        t = torch.tensor([tot], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        tot = float(t.item())
+    h2d = (hq_h.numel() + hk_h.numel() + hv_h.numel()) * 2
+    d2h = out_h.numel() * 2
+    return {"value": round(lay.w.seq_len * args.steps * world / (tot / 1e3), 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(tot / args.steps, 3)}
+
+
+# ----------------------------------------------------------------------------- the CPU oracle
+def oracle_sample(w, n_heads=1, n_rows=32, seed=0):
+    """Times the oracle on a bounded sample of workload w and extrapolates to the
+    layer: per sampled head, the estimation, selection and refinement of every
+    chunk plus the attention of n_rows sampled rows per chunk. Returns
+    (tokens/s, seconds spent, description)."""
+    import oracle.vs_oracle as vo
+
+    st = structure(w)
+    rng = np.random.default_rng(seed)
+    heads = list(range(min(n_heads, w.hq)))
+    dca = (w.dca_chunk, w.dca_window) if w.dca_chunk else None
+    scale = 1.0 / math.sqrt(w.head_dim)
+    t_fixed = 0.0  # per head: estimation + selection/refinement over all chunks
+    t_rows = 0.0  # attention of the sampled rows
+    rows_done = 0
+    spent0 = time.time()
+    for h in heads:
+        hk = h // w.group
+        kf = generate_head(w, "k", hk, st=st).float().double().numpy()
+        vf = generate_head(w, "v", hk, st=st).float().double().numpy()
+        qf = generate_head(w, "q", h, st=st).float().double().numpy()
+        for c in range(w.n_chunks):
+            cs, e = w.chunk_bounds(c)
+            nr = min(w.last_q, e - cs)
+            t0 = time.time()
+            _, vert, slash, a = vo.estimate(qf[e - nr : e], kf, e, w.rope_base, scale)
+            if w.refine_tau is None:
+                V, S = vo.select(vert, slash, w.kv_budget, w.ks_budget)
+            else:
+                _, _, V, S, _, _ = vo.refine(a, np.arange(e - nr, e), vert, slash, w.kv_budget, w.ks_budget,
+                                             w.refine_tau)
+            t1 = time.time()
+            rows = np.sort(rng.choice(np.arange(cs, e), size=min(n_rows, e - cs), replace=False))
+            vo.attention_rows(qf[rows], rows, kf, vf, e, vo.membership(e, V), vo.membership(e, S), w.rope_base,
+                              scale, dca)
+            t2 = time.time()
+            t_fixed += t1 - t0
+            # extrapolate the sampled rows to the chunk's rows
+            t_rows += (t2 - t1) * (e - cs) / len(rows)
+            rows_done += len(rows)
+    per_head = (t_fixed + t_rows) / len(heads)
+    layer_s = per_head * w.hq
+    desc = (f"{len(heads)} of {w.hq} heads; per head all {w.n_chunks} chunks' estimation+selection"
+            f"{'+refinement' if w.refine_tau else ''} and {n_rows} sampled query rows per chunk, extrapolated "
+            f"to every row and head")
+    return w.seq_len / layer_s, time.time() - spent0, desc
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count()
+
+
+def run_reference(args):
+    w = WORKLOADS[args.config]
+    for _ in range(args.warmup):
+        oracle_sample(w, n_heads=1, n_rows=8, seed=99)
+    vals = []
+    for i in range(args.steps):
+        v, spent, desc = oracle_sample(w, n_heads=1, n_rows=16, seed=i)
+        vals.append(v)
+    value = statistics.median(vals)
+    cb = {"value": round(value, 3), "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle", "sample": desc}
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(w.seq_len / value * 1e3, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded generator)",
+        "config": {"workload": w.name, "seq_len": w.seq_len, "hq": w.hq, "hkv": w.hkv},
+        "cpu_baseline": cb,
+        "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ----------------------------------------------------------------------------- main
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return 0
+    if not torch.cuda.is_available():
+        print(json.dumps({"metric": METRIC, "error": "no CUDA device"}))
+        return 1
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    res, w, lay = run_ours(args, rank, world, device)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n_heads, n_rows = (1, 16)
+        v, spent, desc = oracle_sample(w, n_heads=n_heads, n_rows=n_rows)
+        res["cpu_baseline"] = {"value": round(v, 3), "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
+                               "sample": desc, "seconds": round(spent, 1)}
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

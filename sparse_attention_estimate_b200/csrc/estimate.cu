@@ -1,0 +1,492 @@
+// estimate.cu - estimation of the vertical-slash pattern and the recall
+// histogram of sparsity refinement, on tcgen05 tensor cores.
+//
+// Qwen2.5-1M explainer: "Sparse Attention" step 2 (attention of the last
+// queries against all keys), "Chunked Prefill" (the last 64 queries of each
+// chunk), "Algorithm" (selection with continuous positions), "Sparsity
+// Refinement" (attention recall = exp(lse_sparse - lse_full)).
+//
+// One CTA handles one KV head's group (g query heads x 64 estimation rows,
+// tiled as M = 128-row MMA tiles holding two heads each) over a contiguous
+// range of 128-key blocks. Warp 0 issues TMA loads of rotated K blocks into a
+// two-stage ring, warp 1 issues S = Q K^T (tcgen05.mma, M=128 N=128 K=16 bf16,
+// fp32 accumulators in TMEM, one 128-column region per M tile), and two
+// warpgroups (warps 4-7 and 8-11, each thread one TMEM lane = one query row)
+// read S back with tcgen05.ld and run the epilogue of the pass:
+//   kLse    running row max / sum of exp2 -> per-split partials, combined
+//           afterwards into lse (natural log)
+//   kSums   A = exp(s - lse); column sums (vertical) with a warp transpose-sum;
+//           diagonal sums (slash) by rotating each lane's 32 values by its lane
+//           index, splitting wrapped / unwrapped parts and transpose-summing
+//           both; written as per-(head, 32-row half) partial arrays that a fixup
+//           kernel adds in a fixed order (deterministic, no atomics)
+//   kRecall A = exp(s - lse) binned by the first refinement level that selects
+//           the element (min of its column's and its offset's level)
+#include <algorithm>
+#include <cmath>
+
+#include "internal.cuh"
+
+namespace vs {
+
+enum EstMode { kLse = 0, kSums = 1, kRecall = 2 };
+
+constexpr int kEstThreads = 384;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kSOff = 96;  // index offset of the slash partial arrays (skew >= -95)
+
+struct EstParams {
+  int64_t e;          // visible keys
+  int64_t row0;       // position of estimation row 0 (= e - nr)
+  int64_t e_pad;      // row stride of the partial arrays
+  int nr;             // estimation rows per head
+  int g, ntile, hq;
+  int nblk;           // key blocks in [0, e)
+  int bps;            // key blocks per split
+  float scale_log2;   // softmax_scale * log2(e)
+  float* part_ml;     // kLse: [nsplit][hq*64][2] (max, sum) in log2 units
+  const float* lse;   // kSums / kRecall: [hq][64] natural log
+  float* part_v;      // kSums: [hq][2][e_pad]
+  float* part_s;      // kSums: [hq][2][2][e_pad + 256]
+  const uint8_t* lvl; // kRecall: [hq][2][e_pad]
+  float* hist;        // kRecall: [nsplit][hq][kMaxLevels]
+  int nlev;
+  DevCommon dc;
+};
+
+struct __align__(1024) EstSmem {
+  bf16 q[4][2][kTile * 64];  // [M tile][column half], 128-byte swizzled
+  bf16 k[2][2][kTile * 64];  // [stage][column half]
+  uint64_t q_full, k_full[2], k_empty[2], s_full[4], s_empty[4], drain;
+  uint32_t tmem_base;
+  int abort_word;
+  float red[8][kRecallLevels];
+};
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Lane x ends with the sum over the warp's lanes of v[x] (v is consumed).
+__device__ __forceinline__ float warp_transpose_sum32(float (&v)[32]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int s = 16; s >= 1; s >>= 1) {
+    const bool upper = (lane & s) != 0;
+#pragma unroll
+    for (int i = 0; i < s; ++i) {
+      const float keep = upper ? v[i + s] : v[i];
+      const float send = upper ? v[i] : v[i + s];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, s);
+    }
+  }
+  return v[0];
+}
+
+// v[i] <- v[(i + r) mod 32] for a per-lane r in [0, 32): five conditional rotations.
+__device__ __forceinline__ void rotate_by(float (&v)[32], int r) {
+#pragma unroll
+  for (int b = 0; b < 5; ++b) {
+    const bool on = (r >> b) & 1;
+    const int sh = 1 << b;
+    float t[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) t[i] = on ? v[(i + sh) & 31] : v[i];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = t[i];
+  }
+}
+
+// Bounded wait that ignores the abort word (used to drain in-flight copies).
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint64_t limit) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer_ns() - t0 > limit) break;
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kEstThreads, 1)
+    est_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               EstParams p) {
+  extern __shared__ unsigned char smem_raw[];
+  EstSmem& s = *reinterpret_cast<EstSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = blockIdx.y, split = blockIdx.x;
+  const int b_begin = split * p.bps;
+  const int b_end = min(b_begin + p.bps, p.nblk);
+  const int nb = b_end - b_begin;
+  volatile int* abort_word = &s.abort_word;
+
+  if (tid == 0) {
+    mbar_init(&s.q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.k_full[i], 1);
+      mbar_init(&s.k_empty[i], 1);
+    }
+    for (int t = 0; t < 4; ++t) {
+      mbar_init(&s.s_full[t], 1);
+      mbar_init(&s.s_empty[t], 4);
+    }
+    mbar_init(&s.drain, 1);
+    s.abort_word = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&s.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tbase = s.tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0 && nb > 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      mbar_arrive_expect_tx(&s.q_full, p.ntile * 2 * kTile * 64 * 2);
+      for (int t = 0; t < p.ntile; ++t)
+        for (int hf = 0; hf < 2; ++hf) tma_load_3d(s.q[t][hf], &tmQ, &s.q_full, hf * 64, t * kTile, G);
+      int issued[2] = {0, 0};
+      bool ok = true;
+      for (int i = 0; i < nb && ok; ++i) {
+        const int st = i & 1;
+        if (i >= 2) ok = mbar_wait(&s.k_empty[st], ((i >> 1) - 1) & 1, abort_word, p.dc.err);
+        if (!ok) break;
+        mbar_arrive_expect_tx(&s.k_full[st], 2 * kTile * 64 * 2);
+        const int kb = b_begin + i;
+        tma_load_3d(s.k[st][0], &tmK, &s.k_full[st], 0, kb * kTile, G);
+        tma_load_3d(s.k[st][1], &tmK, &s.k_full[st], 64, kb * kTile, G);
+        ++issued[st];
+      }
+      if (!ok) {  // let every issued copy land before the CTA exits
+        drain_wait(&s.q_full, 0, p.dc.wait_ns);
+        for (int st = 0; st < 2; ++st)
+          if (issued[st] > 0) drain_wait(&s.k_full[st], (issued[st] - 1) & 1, p.dc.wait_ns);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && nb > 0) {
+      const uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);
+      bool ok = mbar_wait(&s.q_full, 0, abort_word, p.dc.err);
+      tc_fence_after_sync();
+      for (int i = 0; i < nb && ok; ++i) {
+        const int st = i & 1;
+        ok = mbar_wait(&s.k_full[st], (i >> 1) & 1, abort_word, p.dc.err);
+        if (!ok) break;
+        tc_fence_after_sync();
+        for (int t = 0; t < p.ntile && ok; ++t) {
+          if (i >= 1) ok = mbar_wait(&s.s_empty[t], (i - 1) & 1, abort_word, p.dc.err);
+          if (!ok) break;
+          tc_fence_after_sync();
+          const uint32_t dt = tbase + t * kTile;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * (kTile * 64 * 2) + (kk & 3) * 32;
+            const uint64_t da = smem_desc_sw128(smem_u32(&s.q[t][0][0]) + off, 16, 1024);
+            const uint64_t db = smem_desc_sw128(smem_u32(&s.k[st][0][0]) + off, 16, 1024);
+            mma_bf16_ss(dt, da, db, idesc, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&s.s_full[t]);
+        }
+        mma_commit(&s.k_empty[st]);
+      }
+      // all issued MMAs complete before TMEM is released
+      mma_commit(&s.drain);
+      drain_wait(&s.drain, 0, p.dc.wait_ns);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ epilogue warpgroups
+    const int wg = (warp - 4) >> 2;  // 0 or 1
+    const int wl = warp & 3;         // TMEM lane quarter
+    const int m = wl * 32 + lane;    // row within the M tile
+    const int r = m & 63;            // estimation row within the head
+    const int half = wl & 1;         // 32-row half of the head
+    float st_m[2] = {-INFINITY, -INFINITY}, st_l[2] = {0.f, 0.f};
+    float lse2[2] = {0.f, 0.f};
+    float acc[2][kRecallLevels];
+#pragma unroll
+    for (int a = 0; a < 2; ++a)
+#pragma unroll
+      for (int t = 0; t < kRecallLevels; ++t) acc[a][t] = 0.f;
+#pragma unroll
+    for (int a = 0; a < 2; ++a) {
+      const int t = wg + 2 * a;
+      const int hh = 2 * t + (m >> 6);
+      if (MODE != kLse && t < p.ntile && hh < p.g && r < p.nr)
+        lse2[a] = p.lse[(G * p.g + hh) * kEstRows + r] * kLog2e;
+    }
+    const int64_t irow = p.row0 + r;  // absolute position of this row
+    bool ok = true;
+    for (int i = 0; i < nb && ok; ++i) {
+      const int kb = b_begin + i;
+#pragma unroll
+      for (int a = 0; a < 2; ++a) {
+        const int t = wg + 2 * a;
+        if (t >= p.ntile) break;
+        const int hh = 2 * t + (m >> 6);  // warp-uniform
+        const bool head_ok = hh < p.g;
+        const bool row_ok = head_ok && r < p.nr;
+        const int h = G * p.g + hh;
+        ok = __all_sync(0xffffffffu, mbar_wait(&s.s_full[t], i & 1, abort_word, p.dc.err));
+        if (!ok) break;
+        tc_fence_after_sync();
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t raw[32];
+          tmem_ld32(tmem_addr(tbase + t * kTile, wl * 32, c * 32), raw);
+          tmem_wait_ld();
+          if (c == 3) {
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.s_empty[t]);
+          }
+          const int64_t j0 = static_cast<int64_t>(kb) * kTile + c * 32;
+          float v[32];
+          if (MODE == kLse) {
+            float mx = -INFINITY;
+#pragma unroll
+            for (int x = 0; x < 32; ++x) {
+              const bool valid = row_ok && (j0 + x <= irow);
+              v[x] = valid ? __uint_as_float(raw[x]) * p.scale_log2 : -INFINITY;
+              mx = fmaxf(mx, v[x]);
+            }
+            const float mnew = fmaxf(st_m[a], mx);
+            if (mnew != -INFINITY) {
+              float sum = 0.f;
+#pragma unroll
+              for (int x = 0; x < 32; ++x) sum += ex2(v[x] - mnew);
+              st_l[a] = st_l[a] * ex2(st_m[a] - mnew) + sum;
+              st_m[a] = mnew;
+            }
+          } else {
+#pragma unroll
+            for (int x = 0; x < 32; ++x) {
+              const bool valid = row_ok && (j0 + x <= irow);
+              v[x] = valid ? ex2(__uint_as_float(raw[x]) * p.scale_log2 - lse2[a]) : 0.f;
+            }
+            if (MODE == kSums) {
+              if (head_ok) {
+                // slash: lane l holds row r0 + l; rotate so register i holds column i + l
+                float lo[32], hi[32];
+#pragma unroll
+                for (int x = 0; x < 32; ++x) lo[x] = v[x];
+                rotate_by(lo, lane);
+#pragma unroll
+                for (int x = 0; x < 32; ++x) {
+                  const bool wrapped = x + lane >= 32;
+                  hi[x] = wrapped ? lo[x] : 0.f;
+                  lo[x] = wrapped ? 0.f : lo[x];
+                }
+                const float vs = warp_transpose_sum32(v);
+                const float los = warp_transpose_sum32(lo);
+                const float his = warp_transpose_sum32(hi);
+                const int64_t r0 = half * 32;
+                p.part_v[(static_cast<int64_t>(h) * 2 + half) * p.e_pad + j0 + lane] = vs;
+                float* ps = p.part_s + (static_cast<int64_t>(h) * 2 + half) * 2 * (p.e_pad + 256);
+                ps[j0 + lane - r0 + kSOff] = los;
+                ps[(p.e_pad + 256) + j0 + lane - 32 - r0 + kSOff] = his;
+              }
+            } else {  // kRecall
+              if (row_ok) {
+                const uint8_t* lv_v = p.lvl + static_cast<int64_t>(h) * 2 * p.e_pad;
+                const uint8_t* lv_s = lv_v + p.e_pad;
+#pragma unroll
+                for (int x = 0; x < 32; ++x) {
+                  const int64_t j = j0 + x;
+                  if (j <= irow) {
+                    const int lvv = __ldg(lv_v + j);
+                    const int lvs = __ldg(lv_s + (irow - j));
+                    const int lv = lvv < lvs ? lvv : lvs;
+#pragma unroll
+                    for (int t2 = 0; t2 < kRecallLevels; ++t2) acc[a][t2] += (lv == t2) ? v[x] : 0.f;
+                  }
+                }
+              }
+            }
+          }
+        }
+      }
+    }
+    // ---------------------------------------------------------- per-split outputs
+    if (MODE == kLse) {
+#pragma unroll
+      for (int a = 0; a < 2; ++a) {
+        const int t = wg + 2 * a;
+        const int hh = 2 * t + (m >> 6);
+        if (t < p.ntile && hh < p.g && r < p.nr) {
+          float* o = p.part_ml + ((static_cast<int64_t>(split) * p.hq + G * p.g + hh) * kEstRows + r) * 2;
+          o[0] = st_m[a];
+          o[1] = st_l[a];
+        }
+      }
+    } else if (MODE == kRecall) {
+      // warp sums per level, then the two 32-row halves of each head in a fixed order
+#pragma unroll
+      for (int a = 0; a < 2; ++a) {
+        const int t = wg + 2 * a;
+#pragma unroll
+        for (int t2 = 0; t2 < kRecallLevels; ++t2) {
+          float x = acc[a][t2];
+#pragma unroll
+          for (int o = 16; o >= 1; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+          acc[a][t2] = x;
+        }
+        // warps 2k and 2k+1 of a warpgroup hold the two halves of one head
+        const int slot = (wg * 4 + wl);
+        if (lane == 0)
+          for (int t2 = 0; t2 < kRecallLevels; ++t2) s.red[slot][t2] = acc[a][t2];
+        asm volatile("bar.sync %0, 128;" ::"r"(1 + wg));
+        const int hh = 2 * t + (wl >> 1);
+        if (t < p.ntile && hh < p.g && half == 0 && lane < kRecallLevels) {
+          const float tot = s.red[slot][lane] + s.red[slot + 1][lane];
+          p.hist[(static_cast<int64_t>(split) * p.hq + G * p.g + hh) * kMaxLevels + lane] = tot;
+        }
+        asm volatile("bar.sync %0, 128;" ::"r"(1 + wg));
+      }
+    }
+  }
+  // ------------------------------------------------------------ teardown
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+// lse_i = ln 2 * (max + log2(sum)) over the splits, in split order.
+__global__ void lse_combine_kernel(const float* __restrict__ part_ml, int nsplit, int hq, int nr,
+                                   float* __restrict__ lse) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= hq * kEstRows) return;
+  const int r = idx % kEstRows;
+  if (r >= nr) {
+    lse[idx] = -INFINITY;
+    return;
+  }
+  float mx = -INFINITY;
+  for (int sp = 0; sp < nsplit; ++sp) mx = fmaxf(mx, part_ml[(static_cast<int64_t>(sp) * hq * kEstRows + idx) * 2]);
+  float sum = 0.f;
+  for (int sp = 0; sp < nsplit; ++sp) {
+    const float* q = part_ml + (static_cast<int64_t>(sp) * hq * kEstRows + idx) * 2;
+    if (q[0] != -INFINITY) sum += q[1] * exp2f(q[0] - mx);
+  }
+  lse[idx] = (mx + log2f(sum)) * 0.69314718055994531f;
+}
+
+// vert[j] = sum of the two 32-row halves; slash[d] = the four partial arrays at
+// skew k = row0 - d (lo/hi parts of both halves), each read only where written.
+__global__ void sums_fixup_kernel(const float* __restrict__ part_v, const float* __restrict__ part_s,
+                                  int64_t e, int64_t row0, int64_t e_pad, int64_t cover,
+                                  float* __restrict__ vert, float* __restrict__ slash, int64_t e_ld) {
+  const int h = blockIdx.y;
+  const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (j >= e) return;
+  const float* pv = part_v + static_cast<int64_t>(h) * 2 * e_pad;
+  vert[static_cast<int64_t>(h) * e_ld + j] = pv[j] + pv[e_pad + j];
+  const int64_t d = j;
+  const int64_t k = row0 - d;
+  float acc = 0.f;
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const float* ps = part_s + (static_cast<int64_t>(h) * 2 + half) * 2 * (e_pad + 256);
+    const int64_t r0 = half * 32;
+    // lo array covers skews [-r0, cover-1-r0]; hi covers [-32-r0, cover-33-r0]
+    if (k >= -r0 && k <= cover - 1 - r0) acc += ps[k + kSOff];
+    if (k >= -32 - r0 && k <= cover - 33 - r0) acc += ps[(e_pad + 256) + k + kSOff];
+  }
+  slash[static_cast<int64_t>(h) * e_ld + d] = acc;
+}
+
+static vs_status launch_est(vs_ctx* c, int mode, int64_t e, int nr, const float* lse, int nlev,
+                            int* nsplit_out, cudaStream_t st) {
+  const int hkv = c->cfg.hkv, g = c->cfg.hq / c->cfg.hkv;
+  const int nblk = static_cast<int>(ceil_div(e, kTile));
+  int nsplit = std::max(1, c->num_sms / hkv);
+  nsplit = std::min(nsplit, nblk);
+  nsplit = std::min(nsplit, c->L.nsplit_max);
+  const int bps = static_cast<int>(ceil_div(nblk, nsplit));
+  nsplit = static_cast<int>(ceil_div(nblk, bps));
+  *nsplit_out = nsplit;
+  CUtensorMap tmQ, tmK;
+  vs_status s = make_tmap_rows(&tmQ, c->ws + c->L.q_est, hkv, static_cast<int64_t>(c->L.ntile) * kTile,
+                               static_cast<int64_t>(c->L.ntile) * kTile, kTile);
+  if (s != VS_OK) return s;
+  s = make_tmap_rows(&tmK, c->ws + c->L.k_cont, hkv, e, c->max_seq, kTile);
+  if (s != VS_OK) return s;
+  EstParams p{};
+  p.e = e;
+  p.row0 = e - nr;
+  p.e_pad = c->L.e_pad;
+  p.nr = nr;
+  p.g = g;
+  p.ntile = c->L.ntile;
+  p.hq = c->cfg.hq;
+  p.nblk = nblk;
+  p.bps = bps;
+  p.scale_log2 = c->cfg.softmax_scale * kLog2e;
+  p.part_ml = ws_ptr<float>(c, c->L.est_ml);
+  p.lse = lse;
+  p.part_v = ws_ptr<float>(c, c->L.part_v);
+  p.part_s = ws_ptr<float>(c, c->L.part_s);
+  p.lvl = ws_ptr<uint8_t>(c, c->L.lvl);
+  p.hist = ws_ptr<float>(c, c->L.hist);
+  p.nlev = nlev;
+  p.dc = dev_common(c);
+  const size_t smem = sizeof(EstSmem) + 1024;
+  dim3 grid(nsplit, hkv);
+  cudaError_t err;
+  if (mode == kLse) {
+    cudaFuncSetAttribute(est_kernel<kLse>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    est_kernel<kLse><<<grid, kEstThreads, smem, st>>>(tmQ, tmK, p);
+  } else if (mode == kSums) {
+    cudaFuncSetAttribute(est_kernel<kSums>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    est_kernel<kSums><<<grid, kEstThreads, smem, st>>>(tmQ, tmK, p);
+  } else {
+    cudaFuncSetAttribute(est_kernel<kRecall>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    est_kernel<kRecall><<<grid, kEstThreads, smem, st>>>(tmQ, tmK, p);
+  }
+  (void)err;
+  return launched("est_kernel launch");
+}
+
+vs_status run_estimate(vs_ctx* c, const uint16_t* q, int64_t q_rows, int64_t q_pos0,
+                       const uint16_t* k, int64_t k_rows, int64_t e, float* vert, float* slash,
+                       int64_t e_ld, float* lse, cudaStream_t st) {
+  (void)q;
+  (void)q_rows;
+  (void)k;
+  (void)k_rows;
+  const int nr = static_cast<int>(e - std::max(q_pos0, e - static_cast<int64_t>(c->cfg.last_q)));
+  int nsplit = 0;
+  vs_status s = launch_est(c, kLse, e, nr, nullptr, 0, &nsplit, st);
+  if (s != VS_OK) return s;
+  const int n = c->cfg.hq * kEstRows;
+  lse_combine_kernel<<<ceil_div(n, 256), 256, 0, st>>>(ws_ptr<float>(c, c->L.est_ml), nsplit,
+                                                      c->cfg.hq, nr, lse);
+  s = launched("lse_combine_kernel launch");
+  if (s != VS_OK) return s;
+  s = launch_est(c, kSums, e, nr, lse, 0, &nsplit, st);
+  if (s != VS_OK) return s;
+  const int64_t cover = ceil_div(e, kTile) * kTile;
+  sums_fixup_kernel<<<dim3(static_cast<unsigned>(ceil_div(e, 256)), c->cfg.hq), 256, 0, st>>>(
+      ws_ptr<float>(c, c->L.part_v), ws_ptr<float>(c, c->L.part_s), e, e - nr, c->L.e_pad, cover,
+      vert, slash, e_ld);
+  return launched("sums_fixup_kernel launch");
+}
+
+vs_status run_recall_hist(vs_ctx* c, int64_t e, int nr, const float* lse, int nlev,
+                          cudaStream_t st) {
+  int nsplit = 0;
+  vs_status s = launch_est(c, kRecall, e, nr, lse, nlev, &nsplit, st);
+  c->hist_nsplit = nsplit;
+  return s;
+}
+
+}  // namespace vs

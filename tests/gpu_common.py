@@ -1,0 +1,79 @@
+"""Shared helpers of the GPU parity tests: inputs, conversions, tolerances."""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+import oracle.vs_oracle as vo
+import sparse_attention_estimate_b200 as vsb
+from workloads import generate_layer
+
+# attention outputs (bf16): the spec agreement criteria
+OUT_MAX_ABS = 2e-2
+OUT_MEAN_ABS = 2e-3
+# selection near-ties: candidates within this relative distance of the k-th score
+NEAR_TIE_REL = 1e-4
+# refinement decisions this close to tau may go either way
+TAU_SLACK = 1e-5
+
+
+def f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().double().numpy()
+
+
+def layer_inputs(w, device="cuda"):
+    lay = generate_layer(w)
+    cpu = {k: f64(lay[k]) for k in ("q", "k", "v")}
+    dev = {k: lay[k].to(device) for k in ("q", "k", "v")}
+    return dev, cpu
+
+
+def make_ctx(w, max_chunk=None, dca=None, **kw):
+    C, W = dca if dca is not None else (w.dca_chunk, w.dca_window)
+    cfg = vsb.Config(hq=w.hq, hkv=w.hkv, rope_base=w.rope_base, last_q=w.last_q, dca_chunk=C,
+                     dca_window=W, **kw)
+    return vsb.Context(cfg, max_seq=w.seq_len, max_chunk=max_chunk or min(w.chunk, w.seq_len))
+
+
+def sets_to_lists(sets):
+    v_idx, v_cnt, s_off, s_cnt = [t.cpu().numpy() for t in sets]
+    V = [v_idx[h, : v_cnt[h]].astype(np.int64) for h in range(v_idx.shape[0])]
+    S = [s_off[h, : s_cnt[h]].astype(np.int64) for h in range(s_off.shape[0])]
+    return V, S
+
+
+def lists_to_sets(V, S, cap_v, cap_s, device="cuda"):
+    hq = len(V)
+    v_idx = np.zeros((hq, cap_v), np.int32)
+    s_off = np.zeros((hq, cap_s), np.int32)
+    for h in range(hq):
+        v_idx[h, : len(V[h])] = V[h]
+        s_off[h, : len(S[h])] = S[h]
+    t = lambda a: torch.from_numpy(a).to(device)
+    return (t(v_idx), t(np.array([len(x) for x in V], np.int32)), t(s_off),
+            t(np.array([len(x) for x in S], np.int32)))
+
+
+def assert_near_tie_equal(got, want, score, k):
+    """got/want index sets of the top-k of `score` (float64): they may differ only in
+    elements whose score lies within NEAR_TIE_REL of the k-th score."""
+    got, want = set(map(int, got)), set(map(int, want))
+    if got == want:
+        return
+    kth = vo.kth_score(score, k)
+    tol = NEAR_TIE_REL * abs(kth) + 1e-30
+    for j in got ^ want:
+        s = score[j]
+        assert abs(s - kth) <= tol or (np.isinf(s) and np.isinf(kth)), (j, s, kth)
+
+
+def assert_outputs_close(got: np.ndarray, want: np.ndarray, what=""):
+    d = np.abs(got - want)
+    assert d.max() <= OUT_MAX_ABS, f"{what} max abs {d.max():.3e}"
+    assert d.mean() <= OUT_MEAN_ABS, f"{what} mean abs {d.mean():.3e}"
+
+
+def scale_of(w):
+    return 1.0 / math.sqrt(w.head_dim)

