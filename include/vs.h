@@ -177,6 +177,29 @@ VS_API vs_status vs_prefill_stats(vs_ctx* ctx, cudaStream_t stream, int64_t* out
  * attention kernel, on the call's stream (pass NULL, NULL to stop). */
 VS_API vs_status vs_set_prefill_events(vs_ctx* ctx, cudaEvent_t start, cudaEvent_t stop);
 
+/*
+ * vs_select_noalloc - the selection of vs_select for callers that cannot
+ * allocate device memory. (The paper has no counterpart: this is a deployment
+ * variant of vs_select, not a step of the method.)
+ *
+ * Who needs it: code that may not create a workspace, e.g. a plugin running
+ * inside an application that owns all device memory through its own arena, or
+ * a service that plans its memory at start-up and allows no later cudaMalloc.
+ * It takes no context: hq query heads, vert/slash [hq][e_ld] fp32, budgets and
+ * outputs exactly as in vs_select, except that cap_v and cap_s must be >= e.
+ * Scratch (thresholds and per-element levels) lives in a static device array
+ * of 32 MiB per device, held by every GPU that loads the library until exit;
+ * hq * 2 * round_up(e, 128) bytes plus ~hq * 512 bytes must fit, else
+ * VS_ERR_UNSUPPORTED. Nothing is allocated. The first call on a device looks up
+ * the array's device address (make it before any stream capture begins). Calls
+ * on one device share the array: calls whose kernels overlap on the GPU race.
+ */
+VS_API vs_status vs_select_noalloc(int32_t hq, const float* vert, const float* slash,
+                                   int64_t e_ld, int64_t e, const int32_t* kv_budget,
+                                   const int32_t* ks_budget, int32_t* v_idx, int32_t cap_v,
+                                   int32_t* v_cnt, int32_t* s_off, int32_t cap_s, int32_t* s_cnt,
+                                   cudaStream_t stream);
+
 /* Number of kernels this library has launched in the process so far. */
 VS_API uint64_t vs_kernel_launches(void);
 

@@ -306,4 +306,21 @@ vs_status run_refine_decide(vs_ctx* c, int64_t e, int nr, int nlev, float tau, i
   return launched("refine_decide_kernel launch");
 }
 
+// The three selection kernels on caller-given scratch pointers (no context):
+// thr [hq][2][kMaxLevels][2] uint32, lvl [hq][2][e_pad] uint8, err one int.
+vs_status launch_select_raw(int hq, const float* vert, const float* slash, int64_t e_ld, int64_t e,
+                            const int32_t* kv, const int32_t* ks, uint32_t* thr, uint8_t* lvl,
+                            int64_t e_pad, int* err, int32_t* v_idx, int32_t cap_v, int32_t* v_cnt,
+                            int32_t* s_off, int32_t cap_s, int32_t* s_cnt, cudaStream_t st) {
+  thresholds_kernel<<<dim3(hq, 2), 1024, 0, st>>>(vert, slash, e_ld, e, kv, ks, 1, thr);
+  vs_status s = launched("thresholds_kernel launch");
+  if (s != VS_OK) return s;
+  levels_kernel<<<dim3(hq, 2), 1024, 0, st>>>(vert, slash, e_ld, e, 1, thr, lvl, e_pad);
+  s = launched("levels_kernel launch");
+  if (s != VS_OK) return s;
+  compact_kernel<<<dim3(hq, 2), 1024, 0, st>>>(lvl, e_pad, e, nullptr, v_idx, cap_v, v_cnt, s_off,
+                                              cap_s, s_cnt, err);
+  return launched("compact_kernel launch");
+}
+
 }  // namespace vs

@@ -1,0 +1,90 @@
+// select_noalloc.cu - vs_select_noalloc: the vertical-slash selection of
+// vs_select for callers that cannot allocate device memory.
+//
+// Some callers cannot hand this library a workspace: a plugin loaded into a
+// host application that owns every byte of device memory through its own
+// arena, or a service that plans its memory once at start-up and refuses any
+// later cudaMalloc. vs_select needs a context whose workspace holds the
+// selection thresholds and per-element levels; this entry point keeps that
+// scratch instead in one file-scope device array, so the caller passes only
+// inputs and outputs and nothing is allocated at call time.
+//
+// The array lives in the module image: every GPU that loads the library holds
+// kNoAllocScratchBytes of it until the process exits. Its host-side name is
+// only a stand-in, so its device address is fetched with cudaGetSymbolAddress,
+// once per device, the first time this entry point runs with that device
+// current (make that first call before any stream capture begins). All calls
+// share the array and it keeps the last call's contents; the kernels overwrite
+// every byte they read, so nothing needs clearing, but two calls on one device
+// whose kernels overlap on the GPU (for example on two streams) race on it:
+// serialise them. Each device has its own copy of the array.
+#include <mutex>
+
+#include "internal.cuh"
+
+namespace vs {
+
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB per device
+constexpr int kNoAllocMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_select_scratch[kNoAllocScratchBytes];
+
+vs_status launch_select_raw(int hq, const float* vert, const float* slash, int64_t e_ld, int64_t e,
+                            const int32_t* kv, const int32_t* ks, uint32_t* thr, uint8_t* lvl,
+                            int64_t e_pad, int* err, int32_t* v_idx, int32_t cap_v, int32_t* v_cnt,
+                            int32_t* s_off, int32_t cap_s, int32_t* s_cnt, cudaStream_t st);
+
+// Device address of the scratch array on the current device (looked up once).
+static vs_status scratch_address(unsigned char** out) {
+  static std::mutex mu;
+  static unsigned char* addr[kNoAllocMaxDevices] = {};
+  int dev = -1;
+  vs_status s = cuda_check(cudaGetDevice(&dev), "cudaGetDevice");
+  if (s != VS_OK) return s;
+  if (dev < 0 || dev >= kNoAllocMaxDevices)
+    return set_error(VS_ERR_UNSUPPORTED, "device ordinal %d beyond %d", dev, kNoAllocMaxDevices);
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    s = cuda_check(cudaGetSymbolAddress(&p, g_select_scratch), "cudaGetSymbolAddress(scratch)");
+    if (s != VS_OK) return s;
+    addr[dev] = static_cast<unsigned char*>(p);
+  }
+  *out = addr[dev];
+  return VS_OK;
+}
+
+}  // namespace vs
+
+using namespace vs;
+
+extern "C" vs_status vs_select_noalloc(int32_t hq, const float* vert, const float* slash,
+                                       int64_t e_ld, int64_t e, const int32_t* kv_budget,
+                                       const int32_t* ks_budget, int32_t* v_idx, int32_t cap_v,
+                                       int32_t* v_cnt, int32_t* s_off, int32_t cap_s,
+                                       int32_t* s_cnt, cudaStream_t stream) {
+  if (hq < 1) return set_error(VS_ERR_INVALID_ARG, "hq must be positive");
+  if (!vert || !slash || !kv_budget || !ks_budget || !v_idx || !v_cnt || !s_off || !s_cnt)
+    return set_error(VS_ERR_INVALID_ARG, "a pointer argument is NULL");
+  if (e < 1 || e_ld < e) return set_error(VS_ERR_INVALID_ARG, "need 1 <= e <= e_ld");
+  if (cap_v < e || cap_s < e)
+    return set_error(VS_ERR_INVALID_ARG, "caps must hold e entries (cap_v, cap_s >= e)");
+  // scratch: thresholds, one error word, per-element levels of both arrays
+  const int64_t e_pad = round_up(e, kTile);
+  const size_t thr_bytes = round_up(static_cast<int64_t>(hq) * 2 * kMaxLevels * 2 * 4, 256);
+  const size_t err_bytes = 256;
+  const size_t lvl_bytes = static_cast<size_t>(hq) * 2 * static_cast<size_t>(e_pad);
+  const size_t need = thr_bytes + err_bytes + lvl_bytes;
+  if (need > kNoAllocScratchBytes)
+    return set_error(VS_ERR_UNSUPPORTED,
+                     "hq=%d, e=%lld needs %zu bytes of selection scratch; the no-alloc scratch "
+                     "holds %zu bytes (use vs_select with a context workspace)",
+                     hq, (long long)e, need, kNoAllocScratchBytes);
+  unsigned char* base = nullptr;
+  vs_status s = scratch_address(&base);
+  if (s != VS_OK) return s;
+  return launch_select_raw(hq, vert, slash, e_ld, e, kv_budget, ks_budget,
+                           reinterpret_cast<uint32_t*>(base), base + thr_bytes + err_bytes, e_pad,
+                           reinterpret_cast<int*>(base + thr_bytes), v_idx, cap_v, v_cnt, s_off,
+                           cap_s, s_cnt, stream);
+}
