@@ -61,6 +61,25 @@ def parse():
     return p.parse_args()
 
 
+def rank_workload(w, rank: int):
+    """Rank r > 0 prefills an independent layer: same shapes, seed offset by 1000 r."""
+    return w if rank == 0 else replace(w, seed=w.seed + 1000 * rank)
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """Largest value over the ranks (the job's time is its slowest rank's)."""
+    if world == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(seq_len: int, steps: int, world: int, total_ms: float) -> float:
+    """Whole-job tokens/s: every rank prefilled `steps` layers of seq_len tokens."""
+    return seq_len * steps * world / (total_ms / 1e3)
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -212,9 +231,7 @@ def run_ours(args, rank, world, device):
 
     vsbuild.build()
     vsb.load_library()
-    w = WORKLOADS[args.config]
-    if rank > 0:
-        w = replace(w, seed=w.seed + 1000 * rank)
+    w = rank_workload(WORKLOADS[args.config], rank)
     lay = Layer(w, device, args.max_iters)
     l2 = torch.empty(256 << 20, dtype=torch.uint8, device=device)  # > 126 MB L2
     nchunks = len(lay.chunks)
@@ -259,14 +276,9 @@ def run_ours(args, rank, world, device):
     assert lay.ctx.status() == vsb.VS_OK, "device error in the timed region"
     step_ms = [a.elapsed_time(b) for a, b in step_ev]
     attn_ms = [sum(a.elapsed_time(b) for a, b in evs) for evs in attn_ev]
-    tot_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([tot_ms], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        tot_ms = float(t.item())
+    tot_ms = max_over_ranks(sum(step_ms), world, device)
     ms_per_step = tot_ms / args.steps
-    tokens = w.seq_len * args.steps * world
-    value = tokens / (tot_ms / 1e3)
+    value = job_throughput(w.seq_len, args.steps, world, tot_ms)
     attn_ms_step = sum(attn_ms) / args.steps
     exec_flops = executed * FLOP_PER_TILE
     useful_flops = useful * 4 * 128
@@ -345,14 +357,10 @@ def run_e2e(args, lay, l2, world, device):
         e2e_step()
         evs[i][1].record()
     torch.cuda.synchronize()
-    tot = sum(a.elapsed_time(b) for a, b in evs)
-    if world > 1:
-        t = torch.tensor([tot], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        tot = float(t.item())
+    tot = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), world, device)
     h2d = (hq_h.numel() + hk_h.numel() + hv_h.numel()) * 2
     d2h = out_h.numel() * 2
-    return {"value": round(lay.w.seq_len * args.steps * world / (tot / 1e3), 1), "unit": "tokens/s",
+    return {"value": round(job_throughput(lay.w.seq_len, args.steps, world, tot), 1), "unit": "tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(tot / args.steps, 3)}
 
 

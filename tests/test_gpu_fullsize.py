@@ -41,9 +41,10 @@ def _gpu():
     vsb.load_library()
 
 
-def _run_gpu(w):
-    """The chunk loop of bench.py on device-resident inputs; returns per-chunk
-    host copies of what the checks need."""
+def _run_gpu(w, check_chunks):
+    """The chunk loop of bench.py (estimate -> select/refine -> sparse prefill per
+    chunk) on device-resident inputs; returns host copies of what the checks of
+    the chunks in `check_chunks` need, and the whole output."""
     st = structure(w)
     dev = "cuda"
     q = torch.empty(w.hq, w.seq_len, 128, dtype=torch.bfloat16, device=dev)
@@ -55,28 +56,38 @@ def _run_gpu(w):
     cfg = vsb.Config(hq=w.hq, hkv=w.hkv, rope_base=w.rope_base, last_q=w.last_q, dca_chunk=w.dca_chunk,
                      dca_window=w.dca_window)
     ctx = vsb.Context(cfg, max_seq=w.seq_len, max_chunk=min(w.chunk, w.seq_len))
-    keep = []
-    out = vsb.layer_prefill(ctx, q, k, v, chunk=w.chunk, kv_budget=w.kv_budget, ks_budget=w.ks_budget,
-                            tau=w.refine_tau, keep=keep)
+    out = torch.empty_like(q)
+    lse_o = torch.empty(w.hq, w.seq_len, dtype=torch.float32, device=dev)
+    res = {}
+    for c in range(w.n_chunks):
+        cs, e = w.chunk_bounds(c)
+        vert, slash, lse = ctx.estimate(q, cs, k, e, full=True)
+        kv = torch.full((w.hq,), w.kv_budget, dtype=torch.int32, device=dev)
+        ks = torch.full((w.hq,), w.ks_budget, dtype=torch.int32, device=dev)
+        recall = None
+        if w.refine_tau is None:
+            sets = ctx.select(vert, slash, e, kv, ks)
+        else:
+            sets, recall = ctx.refine(q, cs, k, e, vert, slash, lse, w.refine_tau, kv, ks, full=True)
+        ctx.sparse_prefill(q, cs, e, k, v, sets, out=out, lse=lse_o, full=True)
+        if c in check_chunks:
+            res[c] = dict(cs=cs, e=e, vert=vert.cpu(), slash=slash.cpu(), kv=kv.cpu().numpy(),
+                          ks=ks.cpu().numpy(), recall=None if recall is None else recall.cpu().numpy(),
+                          sets=sets_to_lists(sets), lse=lse_o[:, cs:e].cpu())
+        del vert, slash, lse, sets
     torch.cuda.synchronize()
     assert ctx.status() == vsb.VS_OK
-    res = []
-    for kc in keep:
-        res.append(dict(cs=kc["cs"], e=kc["e"], vert=kc["vert"].cpu(), slash=kc["slash"].cpu(),
-                        kv=kc["kv"].cpu().numpy(), ks=kc["ks"].cpu().numpy(),
-                        recall=None if kc["recall"] is None else kc["recall"].cpu().numpy(),
-                        sets=sets_to_lists(kc["sets"]), lse=kc["lse"].cpu()))
-    return res, out.cpu(), st
+    return res, out, st
 
 
 @pytest.mark.parametrize("cfg", [1, 2, 3, 4, 5])
 def test_fullsize_workload(cfg):
     w = WORKLOADS[cfg]
     chunks_sel, heads_sel, nrows = PLAN[cfg]
-    res, out, st = _run_gpu(w)
+    chunks = list(range(w.n_chunks)) if chunks_sel is None else chunks_sel
+    res, out, st = _run_gpu(w, set(chunks))
     scale = 1.0 / math.sqrt(w.head_dim)
     dca = (w.dca_chunk, w.dca_window) if w.dca_chunk else None
-    chunks = range(w.n_chunks) if chunks_sel is None else chunks_sel
     heads = range(w.hq) if heads_sel is None else heads_sel
     rng = np.random.default_rng(w.seed + 1000)
     kcache = {}
@@ -127,6 +138,6 @@ def test_fullsize_workload(cfg):
             # attention of the sampled rows with the GPU's sets
             oo, ol = vo.attention_rows(q_rows, rows, kf, vf, e, vo.membership(e, V[h]), vo.membership(e, S[h]),
                                        w.rope_base, scale, dca)
-            got = f64(out[h, rows])
+            got = f64(out[h][torch.as_tensor(rows, device=out.device)])
             assert_outputs_close(got, oo, f"cfg{cfg} chunk {c} head {h}")
             assert np.allclose(f64(r["lse"][h, rows - cs]), ol, rtol=0, atol=2e-3), (cfg, c, h)
