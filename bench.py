@@ -58,7 +58,16 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--max-iters", type=int, default=19)
+    p.add_argument("--seq-len", type=int, default=None,
+                   help="prefill only the first SEQ_LEN tokens of the workload (profiling cases)")
     return p.parse_args()
+
+
+def select_workload(args):
+    w = WORKLOADS[args.config]
+    if args.seq_len is not None and args.seq_len < w.seq_len:
+        w = replace(w, seq_len=args.seq_len, name=f"{w.name}_first{args.seq_len}")
+    return w
 
 
 def rank_workload(w, rank: int):
@@ -231,7 +240,7 @@ def run_ours(args, rank, world, device):
 
     vsbuild.build()
     vsb.load_library()
-    w = rank_workload(WORKLOADS[args.config], rank)
+    w = rank_workload(select_workload(args), rank)
     lay = Layer(w, device, args.max_iters)
     l2 = torch.empty(256 << 20, dtype=torch.uint8, device=device)  # > 126 MB L2
     nchunks = len(lay.chunks)
@@ -425,7 +434,7 @@ def cpu_cores():
 
 
 def run_reference(args):
-    w = WORKLOADS[args.config]
+    w = select_workload(args)
     for _ in range(args.warmup):
         oracle_sample(w, n_heads=1, n_rows=8, seed=99)
     vals = []

@@ -20,7 +20,8 @@ from typing import Optional
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libvs.so")
+# the in-tree build; VS_LIBRARY may name another build of the same library
+LIB_PATH = os.environ.get("VS_LIBRARY") or os.path.join(_PKG, "libvs.so")
 
 VS_OK, VS_ERR_INVALID_ARG, VS_ERR_UNSUPPORTED, VS_ERR_WORKSPACE = 0, 1, 2, 3
 VS_ERR_CUDA, VS_ERR_TIMEOUT, VS_ERR_DEVICE_CHECK = 4, 5, 6
@@ -30,7 +31,8 @@ STATUS_NAMES = {0: "VS_OK", 1: "VS_ERR_INVALID_ARG", 2: "VS_ERR_UNSUPPORTED", 3:
 EXPORTS = ("vs_workspace_size", "vs_context_create", "vs_context_destroy", "vs_context_reset",
            "vs_set_wait_limit", "dca_remap", "vs_estimate", "vs_select", "vs_refine",
            "vs_sparse_prefill", "vs_prefill_stats", "vs_status_poll", "vs_selftest_wait_timeout",
-           "vs_last_error", "vs_set_prefill_events", "vs_kernel_launches", "vs_select_noalloc")
+           "vs_last_error", "vs_set_prefill_events", "vs_kernel_launches", "vs_select_noalloc",
+           "vs_selftest_exp2")
 
 
 class VsError(RuntimeError):
@@ -74,6 +76,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "vs_selftest_wait_timeout": [P, U64, P],
         "vs_set_prefill_events": [P, P, P],
         "vs_select_noalloc": [I32, P, P, I64, I64, P, P, P, I32, P, P, I32, P, P],
+        "vs_selftest_exp2": [P, P, I64, P],
     }
     for name, args in sig.items():
         f = getattr(lib, name)

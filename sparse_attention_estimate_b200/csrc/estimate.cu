@@ -304,7 +304,10 @@ __global__ void __launch_bounds__(kEstThreads, 1)
                     const int lvs = __ldg(lv_s + (irow - j));
                     const int lv = lvv < lvs ? lvv : lvs;
 #pragma unroll
-                    for (int t2 = 0; t2 < kRecallLevels; ++t2) acc[a][t2] += (lv == t2) ? v[x] : 0.f;
+                    for (int t2 = 0; t2 < kRecallLevels; ++t2) {
+                      if (t2 >= p.nlev) break;  // uniform: levels in use only
+                      acc[a][t2] += (lv == t2) ? v[x] : 0.f;
+                    }
                   }
                 }
               }

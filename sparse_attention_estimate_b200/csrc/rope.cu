@@ -28,14 +28,16 @@ __device__ __forceinline__ double bf16_bits_to_f64(uint16_t u) {
   return static_cast<double>(__uint_as_float(static_cast<uint32_t>(u) << 16));
 }
 
-// One thread per (row, rotary pair); 4 rows of 64 pairs per 256-thread block.
-// Each thread evaluates its cos/sin once and applies them to every head.
+// One thread per (row, 8 consecutive rotary pairs): 16-byte loads and stores of
+// x[m0..m0+7] and x[m0+64..m0+71]; 32 rows per 256-thread block. Each thread
+// evaluates its 8 cos/sin pairs once and applies them to every head.
+constexpr int kRopePairs = 8;
 __global__ void __launch_bounds__(256) rope_rows_kernel(
     const uint16_t* __restrict__ in, int64_t in_rows, int64_t in_row0, uint16_t* __restrict__ out,
     int64_t out_row0, int gdiv, int64_t gstride, int64_t hstride, int64_t nrows, int nheads,
     int64_t pos0, int mode, DcaParams dca, const double* __restrict__ theta) {
-  const int64_t r = static_cast<int64_t>(blockIdx.x) * 4 + (threadIdx.x >> 6);
-  const int m = threadIdx.x & 63;
+  const int64_t r = static_cast<int64_t>(blockIdx.x) * 32 + (threadIdx.x >> 3);
+  const int m0 = (threadIdx.x & 7) * kRopePairs;
   if (r >= nrows) return;
   const int64_t t = pos0 + r;
   int64_t p;
@@ -45,20 +47,36 @@ __global__ void __launch_bounds__(256) rope_rows_kernel(
     p = dca_key_pos(t, dca);
   else
     p = dca_query_pos(t, mode - 2, dca);
-  const double ang = __dmul_rn(static_cast<double>(p), theta[m]);
-  double s, c;
-  sincos(ang, &s, &c);
+  double s[kRopePairs], c[kRopePairs];
+#pragma unroll
+  for (int q = 0; q < kRopePairs; ++q) sincos(__dmul_rn(static_cast<double>(p), theta[m0 + q]), &s[q], &c[q]);
   for (int h = 0; h < nheads; ++h) {
     const uint16_t* x = in + (static_cast<int64_t>(h) * in_rows + in_row0 + r) * kD;
-    const double x1 = bf16_bits_to_f64(x[m]);
-    const double x2 = bf16_bits_to_f64(x[m + kHalf]);
-    const double y1 = __dsub_rn(__dmul_rn(x1, c), __dmul_rn(x2, s));
-    const double y2 = __dadd_rn(__dmul_rn(x2, c), __dmul_rn(x1, s));
+    const uint4 a = *reinterpret_cast<const uint4*>(x + m0);
+    const uint4 b = *reinterpret_cast<const uint4*>(x + m0 + kHalf);
+    const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+    uint32_t ya[4], yb[4];
+#pragma unroll
+    for (int q2 = 0; q2 < 4; ++q2) {
+      uint32_t lo_a = 0, lo_b = 0;
+#pragma unroll
+      for (int k2 = 0; k2 < 2; ++k2) {
+        const int q = 2 * q2 + k2;
+        const double x1 = bf16_bits_to_f64(static_cast<uint16_t>(wa[q2] >> (16 * k2)));
+        const double x2 = bf16_bits_to_f64(static_cast<uint16_t>(wb[q2] >> (16 * k2)));
+        const uint32_t y1 = f64_to_bf16_rne(__dsub_rn(__dmul_rn(x1, c[q]), __dmul_rn(x2, s[q])));
+        const uint32_t y2 = f64_to_bf16_rne(__dadd_rn(__dmul_rn(x2, c[q]), __dmul_rn(x1, s[q])));
+        lo_a |= y1 << (16 * k2);
+        lo_b |= y2 << (16 * k2);
+      }
+      ya[q2] = lo_a;
+      yb[q2] = lo_b;
+    }
     const int64_t orow = static_cast<int64_t>(h / gdiv) * gstride +
                          static_cast<int64_t>(h % gdiv) * hstride + out_row0 + r;
     uint16_t* y = out + orow * kD;
-    y[m] = f64_to_bf16_rne(y1);
-    y[m + kHalf] = f64_to_bf16_rne(y2);
+    *reinterpret_cast<uint4*>(y + m0) = make_uint4(ya[0], ya[1], ya[2], ya[3]);
+    *reinterpret_cast<uint4*>(y + m0 + kHalf) = make_uint4(yb[0], yb[1], yb[2], yb[3]);
   }
 }
 
@@ -68,7 +86,7 @@ vs_status launch_rope_rows(vs_ctx* c, const bf16* in, int64_t in_rows, int64_t i
                            cudaStream_t st) {
   (void)out_rows;
   if (nrows <= 0) return VS_OK;
-  const int64_t blocks = ceil_div(nrows, 4);
+  const int64_t blocks = ceil_div(nrows, 32);
   rope_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
       reinterpret_cast<const uint16_t*>(in), in_rows, in_row0, reinterpret_cast<uint16_t*>(out),
       out_row0, out_gdiv, out_gstride, out_hstride, nrows, nheads, pos0, mode, c->dca, c->theta);

@@ -10,10 +10,12 @@
 // inputs and outputs and nothing is allocated at call time.
 //
 // The array lives in the module image: every GPU that loads the library holds
-// kNoAllocScratchBytes of it until the process exits. Its host-side name is
-// only a stand-in, so its device address is fetched with cudaGetSymbolAddress,
-// once per device, the first time this entry point runs with that device
-// current (make that first call before any stream capture begins). All calls
+// kNoAllocScratchBytes of it until the process exits (the driver reserves it
+// when the library's device code is loaded; with CUDA's lazy module loading
+// that happens at the first call here). Its host-side name is only a
+// stand-in, so its device address is fetched with cudaGetSymbolAddress, once
+// per device, the first time this entry point runs with that device current
+// (make that first call before any stream capture begins). All calls
 // share the array and it keeps the last call's contents; the kernels overwrite
 // every byte they read, so nothing needs clearing, but two calls on one device
 // whose kernels overlap on the GPU (for example on two streams) race on it:

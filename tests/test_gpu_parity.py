@@ -1,5 +1,7 @@
 """Parity of every library call with the CPU oracle, on small seeded workloads
 that span several 128-row tiles / 128-key blocks and end in ragged tails."""
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -30,6 +32,9 @@ CASES = {
                                     ks_budget=50, refine_tau=0.9), None),
     "g5_dca": (small_workload(5, seq_len=1400, chunk=512, hq=5, hkv=1, n_planted=16, kv_budget=64,
                               ks_budget=96, refine_tau=0.9), (512, 128)),
+    # MHA (group 1: half-empty estimation tile); the last chunk holds a single row
+    "g1_tail1": (small_workload(2, seq_len=641, chunk=640, hq=2, hkv=2, n_planted=4, kv_budget=20,
+                                ks_budget=30, refine_tau=0.9), None),
 }
 
 
@@ -278,3 +283,57 @@ def test_host_validation_on_device():
     bad = lists_to_sets([np.array([0, 600])] * 2, S, 8, 8)
     ctx.sparse_prefill(dev["q"], 0, 512, dev["k"], dev["v"], bad)
     assert ctx.status() == vsb.VS_ERR_DEVICE_CHECK
+
+
+def test_fma_pipe_exp2_within_its_error_bound():
+    """The exp2 the attention kernel evaluates on its FMA pipe for part of the
+    softmax, against float64 exp2: relative error below 1e-4 over its range."""
+    lib = vsb.load_library()
+    rng = np.random.default_rng(17)
+    x = np.concatenate([rng.uniform(-125.0, 16.0, 200000), rng.uniform(-1.0, 1.0, 50000),
+                        np.array([0.0, -0.5, 0.5, 1.0, -1.0, 7.999, 8.0, -124.9, -125.0, 15.5])])
+    x = x[: (len(x) // 2) * 2].astype(np.float32)
+    xd = torch.from_numpy(x).cuda()
+    yd = torch.empty_like(xd)
+    st = lib.vs_selftest_exp2(ctypes.c_void_p(xd.data_ptr()), ctypes.c_void_p(yd.data_ptr()), xd.numel(),
+                              ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == vsb.VS_OK
+    y = yd.cpu().double().numpy()
+    ref = np.exp2(x.astype(np.float64))
+    rel = np.abs(y / ref - 1.0)
+    assert rel.max() < 1e-4, rel.max()
+
+
+def test_dca_with_chunk_beyond_sequence_equals_continuous_rope():
+    """DCA whose chunk covers the sequence reduces to plain RoPE: the GPU path
+    with DCA gives the same outputs as without it (bit-identical)."""
+    w = small_workload(2, seq_len=900, chunk=512, hq=4, hkv=2)
+    dev, _ = layer_inputs(w)
+    V, S = _random_sets(np.random.default_rng(9), w.hq, w.seq_len, 0.2, 0.05)
+    outs = []
+    for dca in (None, (1152, 128)):  # S = 1024 >= 900
+        ctx = make_ctx(w, max_chunk=w.chunk, dca=dca)
+        out = torch.zeros_like(dev["q"])
+        for cs, e in _chunks(w):
+            sets = lists_to_sets([x[x < e] for x in V], [x[x < e] for x in S], e, e)
+            ctx.sparse_prefill(dev["q"], cs, e, dev["k"], dev["v"], sets, out=out, full=True)
+        assert ctx.status() == vsb.VS_OK
+        outs.append(out)
+    assert torch.equal(outs[0], outs[1])
+
+
+def test_empty_and_out_of_range_sizes_are_rejected():
+    w = small_workload(2, seq_len=512, chunk=512, hq=2, hkv=1)
+    dev, _ = layer_inputs(w)
+    ctx = make_ctx(w, max_chunk=256)
+    with pytest.raises(vsb.VsError):
+        ctx.estimate(dev["q"], 0, dev["k"], 0)
+    buf = torch.empty(2, 64, dtype=torch.float32, device="cuda")
+    p = lambda t: ctypes.c_void_p(t.data_ptr())
+    for e in (0, -1, 513):  # empty, negative, beyond max_seq
+        st = ctx.lib.vs_estimate(ctx.handle, p(dev["q"]), 512, 0, p(dev["k"]), 512, e, p(buf), p(buf), 64, p(buf),
+                                 None)
+        assert st in (vsb.VS_ERR_INVALID_ARG, vsb.VS_ERR_UNSUPPORTED), (e, st)
+    with pytest.raises(vsb.VsError):  # a chunk of 512 rows, longer than max_chunk = 256
+        ctx.sparse_prefill(dev["q"], 0, 512, dev["k"], dev["v"], lists_to_sets([np.arange(4)] * 2, [np.arange(1)] * 2, 8, 8))
+    assert ctx.status() == vsb.VS_OK

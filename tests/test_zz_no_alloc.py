@@ -7,6 +7,7 @@ This file is collected last so that a run stopping at the first failure has
 already run every other test; it also passes alone in a fresh process.
 """
 import ctypes
+import gc
 
 import numpy as np
 import pytest
@@ -45,12 +46,25 @@ def test_select_noalloc_matches_select_on_two_calls_in_a_row():
                torch.full((w.hq,), -1, dtype=torch.int32, device="cuda"),
                torch.full((w.hq, e), -1, dtype=torch.int32, device="cuda"),
                torch.full((w.hq,), -1, dtype=torch.int32, device="cuda")]
-        n0 = torch.cuda.memory_allocated()
-        st = lib.vs_select_noalloc(w.hq, _p(vert), _p(slash), vert.stride(0), e, _p(kv), _p(ks), _p(got[0]), e,
-                                   _p(got[1]), _p(got[2]), e, _p(got[3]), stream)
-        assert st == vsb.VS_OK, lib.vs_last_error()
-        torch.cuda.synchronize()
-        assert torch.cuda.memory_allocated() == n0
+        # nothing may be allocated by a call: neither through torch nor on the device.
+        # The first call on a device does the one-time set-up (the address lookup, at
+        # which CUDA's lazy module loading may reserve the static array), so the device
+        # check applies from the second call on. Garbage collection is held off so
+        # earlier tests' tensors are not freed meanwhile.
+        gc.collect()
+        gc.disable()
+        try:
+            torch.cuda.synchronize()
+            n0, free0 = torch.cuda.memory_allocated(), torch.cuda.mem_get_info()[0]
+            st = lib.vs_select_noalloc(w.hq, _p(vert), _p(slash), vert.stride(0), e, _p(kv), _p(ks), _p(got[0]),
+                                       e, _p(got[1]), _p(got[2]), e, _p(got[3]), stream)
+            assert st == vsb.VS_OK, lib.vs_last_error()
+            torch.cuda.synchronize()
+            assert torch.cuda.memory_allocated() == n0
+            if call > 0:
+                assert torch.cuda.mem_get_info()[0] == free0
+        finally:
+            gc.enable()
         assert ctx.status() == vsb.VS_OK
         r_vi, r_vc, r_so, r_sc = [t.cpu() for t in ref]
         g_vi, g_vc, g_so, g_sc = [t.cpu() for t in got]
