@@ -213,12 +213,6 @@ VS_API vs_status vs_status_poll(vs_ctx* ctx, cudaStream_t stream);
  * failure path of every wait without faulting the GPU. */
 VS_API vs_status vs_selftest_wait_timeout(vs_ctx* ctx, uint64_t limit_ns, cudaStream_t stream);
 
-/* Evaluates, for n (even) fp32 inputs x in [-125, 16), the exp2 that the
- * attention kernel runs on its FMA pipe for part of the softmax (round-to-
- * nearest range reduction, a cubic for 2^f on [-1/2, 1/2], exponent add), so
- * tests can hold it to its error bound (relative error < 1e-4). y: n fp32. */
-VS_API vs_status vs_selftest_exp2(const float* x, float* y, int64_t n, cudaStream_t stream);
-
 /* Message of the last error on this thread (never NULL). */
 VS_API const char* vs_last_error(void);
 

@@ -31,8 +31,7 @@ STATUS_NAMES = {0: "VS_OK", 1: "VS_ERR_INVALID_ARG", 2: "VS_ERR_UNSUPPORTED", 3:
 EXPORTS = ("vs_workspace_size", "vs_context_create", "vs_context_destroy", "vs_context_reset",
            "vs_set_wait_limit", "dca_remap", "vs_estimate", "vs_select", "vs_refine",
            "vs_sparse_prefill", "vs_prefill_stats", "vs_status_poll", "vs_selftest_wait_timeout",
-           "vs_last_error", "vs_set_prefill_events", "vs_kernel_launches", "vs_select_noalloc",
-           "vs_selftest_exp2")
+           "vs_last_error", "vs_set_prefill_events", "vs_kernel_launches", "vs_select_noalloc")
 
 
 class VsError(RuntimeError):
@@ -76,7 +75,6 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "vs_selftest_wait_timeout": [P, U64, P],
         "vs_set_prefill_events": [P, P, P],
         "vs_select_noalloc": [I32, P, P, I64, I64, P, P, P, I32, P, P, I32, P, P],
-        "vs_selftest_exp2": [P, P, I64, P],
     }
     for name, args in sig.items():
         f = getattr(lib, name)

@@ -436,12 +436,6 @@ extern "C" vs_status vs_status_poll(vs_ctx* c, cudaStream_t st) {
   return VS_OK;
 }
 
-extern "C" vs_status vs_selftest_exp2(const float* x, float* y, int64_t n, cudaStream_t st) {
-  VS_REQUIRE(x && y, VS_ERR_INVALID_ARG, "x and y must not be NULL");
-  VS_REQUIRE(n >= 0 && n % 2 == 0, VS_ERR_INVALID_ARG, "n must be even and non-negative");
-  return launch_exp2_selftest(x, y, n, st);
-}
-
 extern "C" vs_status vs_selftest_wait_timeout(vs_ctx* c, uint64_t limit_ns, cudaStream_t st) {
   VS_TRY(check_ctx(c));
   VS_REQUIRE(limit_ns >= 1000 && limit_ns <= 10000000000ull, VS_ERR_INVALID_ARG,

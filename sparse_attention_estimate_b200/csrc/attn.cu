@@ -217,30 +217,6 @@ __device__ __forceinline__ float ex2a(float x) {
   return y;
 }
 
-// exp2 of two finite arguments on the FMA pipe (relieves the MUFU pipe):
-// a = n + f with n = round(a) and f in [-1/2, 1/2] (adding 1.5 * 2^23 rounds to
-// an integer held in the low mantissa bits); 2^f from a cubic whose coefficients
-// were fitted here for minimax relative error on [-1/2, 1/2] (Lawson's
-// iteratively reweighted least squares; max relative error 7.5e-5 in fp32,
-// below the 2^-9 of the bf16 probabilities); 2^n is added to the exponent
-// field. Arguments are clamped at -125 so the exponent cannot underflow.
-__device__ __forceinline__ void exp2_poly_pair(float a0, float a1, float& p0, float& p1) {
-  constexpr float kC0 = 0.99992808f, kC1 = 0.69326099f, kC2 = 0.24261094f, kC3 = 0.05517149f;
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  const uint64_t a2 = f32x2_pack(fmaxf(a0, -125.f), fmaxf(a1, -125.f));
-  const uint64_t t2 = f32x2_add(a2, f32x2_pack(kRound, kRound));
-  const uint64_t n2 = f32x2_add(t2, f32x2_pack(-kRound, -kRound));
-  const uint64_t f2 = f32x2_fma(n2, f32x2_pack(-1.f, -1.f), a2);
-  uint64_t q2 = f32x2_fma(f32x2_pack(kC3, kC3), f2, f32x2_pack(kC2, kC2));
-  q2 = f32x2_fma(q2, f2, f32x2_pack(kC1, kC1));
-  q2 = f32x2_fma(q2, f2, f32x2_pack(kC0, kC0));
-  float q0, q1, t0, t1;
-  f32x2_unpack(q2, q0, q1);
-  f32x2_unpack(t2, t0, t1);
-  p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
-  p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
-}
-
 __device__ __forceinline__ void drain_wait_a(uint64_t* bar, uint32_t parity, uint64_t limit) {
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity))
@@ -315,8 +291,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       int kiss[2] = {0, 0}, viss[2] = {0, 0};
       bool ok = true;
+      int32_t ent = list[0];  // schedule entries are read one block ahead of use
       for (int j = 0; j < n && ok; ++j) {
-        const int b = list[j] & 0xFFFFFF;
+        const int b = ent & 0xFFFFFF;
+        ent = j + 1 < n ? ld_keep_s32(list + j + 1) : 0;
         const int st = j & 1;
         // K(j) first: the MMA warp releases a Q tile only after issuing S0(j)
         if (j >= 2) ok = mbar_wait(&s.k_empty[st], ((j >> 1) - 1) & 1, abort_word, p.dc.err);
@@ -368,6 +346,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int64_t kb0 = static_cast<int64_t>(list[0] & 0xFFFFFF) * kTile;
         cls[0] = dca_class(R0, kb0, p.dca);
         cls[1] = dca_class(R0 + kTile, kb0, p.dca);
+        int32_t ent1 = n > 1 ? list[1] : 0;  // entry of block j + 1, read a block ahead
         auto issue_qk = [&](int t, int st) {
           const uint32_t qa = smem_u32(&s.q[t][0][0]);
           const uint32_t ka = smem_u32(&s.k[st][0][0]);
@@ -400,7 +379,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const int st = j & 1;
           const bool more = j + 1 < n;
           const int st1 = (j + 1) & 1;
-          const int64_t kb1 = more ? static_cast<int64_t>(list[j + 1] & 0xFFFFFF) * kTile : 0;
+          const int64_t kb1 = more ? static_cast<int64_t>(ent1 & 0xFFFFFF) * kTile : 0;
+          ent1 = j + 2 < n ? ld_keep_s32(list + j + 2) : 0;
           // tile 0
           ok = mbar_wait(&s.p_full[0], j & 1, abort_word, p.dc.err) &&
                mbar_wait(&s.v_full[st], (j >> 1) & 1, abort_word, p.dc.err);
@@ -458,10 +438,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t* vb = p.vbits + static_cast<int64_t>(h) * p.nwords;
     const uint32_t* sb = p.sbits + static_cast<int64_t>(h) * p.nwords;
     float m_run = -INFINITY, l_run = 0.f;
+    int32_t ent = n > 0 ? list[0] : 0;  // schedule entry of block j, read a block ahead
     unsigned long long useful = 0;
     bool ok = true;
     for (int j = 0; j < n && ok; ++j) {
-      const int32_t entry = list[j];
+      const int32_t entry = ent;
+      ent = j + 1 < n ? ld_keep_s32(list + j + 1) : 0;
       const int64_t k0 = static_cast<int64_t>(entry & 0xFFFFFF) * kTile;
       const int state = (entry >> (24 + 2 * t)) & 3;
       // element mask of this row over the block's 128 keys
@@ -505,31 +487,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&s.s_full[t], j & 1, abort_word, p.dc.err));
       if (!ok) break;
       tc_fence_after_sync();
-      // All 128 scores of the row are loaded with four tcgen05.ld and one wait;
-      // blocks where every lane keeps all 128 keys skip the mask selects. The row
-      // max runs over 8 independent three-input max chains.
-      uint32_t sr[4][32];
+      float sv[128];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
+      for (int c = 0; c < 4; ++c) {
+        uint32_t raw[32];
+        tmem_ld32(tS + c * 32, raw);
+#pragma unroll
+        for (int x = 0; x < 32; ++x) sv[c * 32 + x] = __uint_as_float(raw[x]);
+      }
       tmem_wait_ld();
       const bool all_on = __all_sync(0xffffffffu, (mw[0] & mw[1] & mw[2] & mw[3]) == 0xFFFFFFFFu);
       if (!all_on) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int x = 0; x < 32; ++x)
-            if (!((mw[c] >> x) & 1u)) sr[c][x] = 0xFF800000u;  // -inf
+        for (int c = 0; c < 128; ++c)
+          if (!((mw[c >> 5] >> (c & 31)) & 1u)) sv[c] = -INFINITY;
       }
-      float mx[8];
+      float mx[16];
 #pragma unroll
-      for (int x = 0; x < 8; ++x) mx[x] = -INFINITY;
+      for (int x = 0; x < 16; ++x) mx[x] = fmaxf(sv[x], sv[x + 16]);
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int c = 32; c < 128; c += 16)
 #pragma unroll
-        for (int x = 0; x < 32; x += 2)
-          mx[(x >> 1) & 7] = fmax3(mx[(x >> 1) & 7], __uint_as_float(sr[c][x]), __uint_as_float(sr[c][x + 1]));
-      const float mblk = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) *
-                         p.scale_log2;  // scale > 0 keeps the order
+        for (int x = 0; x < 16; ++x) mx[x] = fmaxf(mx[x], sv[c + x]);
+#pragma unroll
+      for (int w2 = 8; w2 >= 1; w2 >>= 1)
+#pragma unroll
+        for (int x = 0; x < w2; ++x) mx[x] = fmaxf(mx[x], mx[x + w2]);
+      const float mblk = mx[0] * p.scale_log2;
       useful += __popc(mw[0]) + __popc(mw[1]) + __popc(mw[2]) + __popc(mw[3]);
       // lazy rescale: move the reference max only when it grows by > 2^8
       const float m_new = fmaxf(m_run, mblk);
@@ -551,59 +535,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         l_run *= f;
         m_run = m_new;
       }
-      // p = exp2(s * scale * log2(e) - m): the argument of two columns per packed
-      // fp32x2 FMA, one MUFU exp2 per element, the row sum over 4 packed chains.
-      // P goes back as bf16 pairs into the first 64 columns of S, 32 columns of P
-      // (16 TMEM columns) at a time, so only one chunk of packed P is live.
       const float nm = (m_run == -INFINITY) ? 0.f : -m_run;
-      const uint64_t sc2 = f32x2_pack(p.scale_log2, p.scale_log2);
-      const uint64_t nm2 = f32x2_pack(nm, nm);
-      uint64_t ls2[4];
+      float ls[8];
 #pragma unroll
-      for (int x = 0; x < 4; ++x) ls2[x] = 0ull;
+      for (int x = 0; x < 8; ++x) ls[x] = 0.f;
+      uint32_t pk[64];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
-        if (all_on) {
-          // finite arguments only: 5 of every 16 pairs go to the FMA-pipe exp2
-#pragma unroll
-          for (int x = 0; x < 16; ++x) {
-            const uint64_t a2 = f32x2_fma(
-                f32x2_pack(__uint_as_float(sr[c][2 * x]), __uint_as_float(sr[c][2 * x + 1])), sc2, nm2);
-            float a0, a1, p0, p1;
-            f32x2_unpack(a2, a0, a1);
-            if (x % 3 == 2) {
-              exp2_poly_pair(a0, a1, p0, p1);
-            } else {
-              p0 = ex2a(a0);
-              p1 = ex2a(a1);
-            }
-            ls2[x & 3] = f32x2_add(ls2[x & 3], f32x2_pack(p0, p1));
-            pk[x] = pack_bf16x2(p0, p1);
-          }
-        } else {
-          // masked entries are -inf and must give exactly 0: MUFU exp2 only
-#pragma unroll
-          for (int x = 0; x < 16; ++x) {
-            const uint64_t a2 = f32x2_fma(
-                f32x2_pack(__uint_as_float(sr[c][2 * x]), __uint_as_float(sr[c][2 * x + 1])), sc2, nm2);
-            float a0, a1;
-            f32x2_unpack(a2, a0, a1);
-            const float p0 = ex2a(a0), p1 = ex2a(a1);
-            ls2[x & 3] = f32x2_add(ls2[x & 3], f32x2_pack(p0, p1));
-            pk[x] = pack_bf16x2(p0, p1);
-          }
-        }
-        tmem_st16(tS + c * 16, pk);
+      for (int c = 0; c < 64; ++c) {
+        const float p0 = ex2a(fmaf(sv[2 * c], p.scale_log2, nm));
+        const float p1 = ex2a(fmaf(sv[2 * c + 1], p.scale_log2, nm));
+        ls[(2 * c) & 7] += p0;
+        ls[(2 * c + 1) & 7] += p1;
+        pk[c] = pack_bf16x2(p0, p1);
       }
-      float lsum = 0.f;
 #pragma unroll
-      for (int x = 0; x < 4; ++x) {
-        float u0, u1;
-        f32x2_unpack(ls2[x], u0, u1);
-        lsum += u0 + u1;
-      }
-      l_run += lsum;
+      for (int w2 = 4; w2 >= 1; w2 >>= 1)
+#pragma unroll
+        for (int x = 0; x < w2; ++x) ls[x] += ls[x + w2];
+      l_run += ls[0];
+      tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(pk));
+      tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
       tmem_wait_st();
       tc_fence_before_sync();
       __syncwarp();
@@ -732,23 +683,6 @@ vs_status run_sparse_prefill(vs_ctx* c, const uint16_t* q, int64_t q_rows, int64
   s = launched("attn_kernel launch");
   if (s == VS_OK && c->ev_stop) s = cuda_check(cudaEventRecord(c->ev_stop, st), "timing event");
   return s;
-}
-
-// ---------------------------------------------------------------- exp2 self-test
-__global__ void exp2_poly_selftest_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t npairs) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= npairs) return;
-  float p0, p1;
-  exp2_poly_pair(x[2 * i], x[2 * i + 1], p0, p1);
-  y[2 * i] = p0;
-  y[2 * i + 1] = p1;
-}
-
-vs_status launch_exp2_selftest(const float* x, float* y, int64_t n, cudaStream_t st) {
-  const int64_t npairs = n / 2;
-  if (npairs == 0) return VS_OK;
-  exp2_poly_selftest_kernel<<<static_cast<unsigned>(ceil_div(npairs, 256)), 256, 0, st>>>(x, y, npairs);
-  return launched("exp2_poly_selftest_kernel launch");
 }
 
 // ---------------------------------------------------------------- wait self-test

@@ -147,7 +147,6 @@ vs_status run_sparse_prefill(vs_ctx* c, const uint16_t* q, int64_t q_rows, int64
                              const int32_t* s_off, int32_t cap_s, const int32_t* s_cnt,
                              uint16_t* out, float* lse_out, cudaStream_t st);
 vs_status launch_wait_selftest(vs_ctx* c, uint64_t limit_ns, cudaStream_t st);
-vs_status launch_exp2_selftest(const float* x, float* y, int64_t n, cudaStream_t st);
 
 // Counts a kernel launch (vs_kernel_launches) and returns the launch error state.
 vs_status launched(const char* what);
