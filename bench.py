@@ -374,55 +374,69 @@ def run_e2e(args, lay, l2, world, device):
 
 
 # ----------------------------------------------------------------------------- the CPU oracle
-def oracle_sample(w, n_heads=1, n_rows=32, seed=0):
+def oracle_sample(w, budget_s=15.0, n_rows=64, seed=0):
     """Times the oracle on a bounded sample of workload w and extrapolates to the
-    layer: per sampled head, the estimation, selection and refinement of every
-    chunk plus the attention of n_rows sampled rows per chunk. Returns
-    (tokens/s, seconds spent, description)."""
+    layer. Work units are (head, chunk) pairs: the chunk's estimation, selection
+    and refinement for that head, plus the attention of n_rows sampled query rows
+    of the chunk. Units run in a spread order (heads in turn, chunks from the
+    last, longest one down) until budget_s of wall time is spent (at least one
+    unit). Each unit's cost is taken as linear in its key count e (estimation and
+    per-row attention both are), so the measured per-key rates extrapolate to
+    every chunk, row and head. Returns (tokens/s, seconds spent, description)."""
     import oracle.vs_oracle as vo
 
     st = structure(w)
     rng = np.random.default_rng(seed)
-    heads = list(range(min(n_heads, w.hq)))
     dca = (w.dca_chunk, w.dca_window) if w.dca_chunk else None
     scale = 1.0 / math.sqrt(w.head_dim)
-    t_fixed = 0.0  # per head: estimation + selection/refinement over all chunks
-    t_rows = 0.0  # attention of the sampled rows
-    rows_done = 0
+    chunks = list(range(w.n_chunks - 1, -1, -1))
+    units = [(h, c) for c in chunks for h in range(w.hq)]
+    fixed_per_key, row_per_key = [], []  # seconds per key of e: per chunk, and per row and chunk
+    cache = {}
     spent0 = time.time()
-    for h in heads:
+    done = 0
+    for h, c in units:
+        if done and time.time() - spent0 >= budget_s:
+            break
         hk = h // w.group
-        kf = generate_head(w, "k", hk, st=st).float().double().numpy()
-        vf = generate_head(w, "v", hk, st=st).float().double().numpy()
-        qf = generate_head(w, "q", h, st=st).float().double().numpy()
-        for c in range(w.n_chunks):
-            cs, e = w.chunk_bounds(c)
-            nr = min(w.last_q, e - cs)
-            t0 = time.time()
-            _, vert, slash, a = vo.estimate(qf[e - nr : e], kf, e, w.rope_base, scale)
-            if w.refine_tau is None:
-                V, S = vo.select(vert, slash, w.kv_budget, w.ks_budget)
-            else:
-                _, _, V, S, _, _ = vo.refine(a, np.arange(e - nr, e), vert, slash, w.kv_budget, w.ks_budget,
-                                             w.refine_tau)
-            t1 = time.time()
-            rows = np.sort(rng.choice(np.arange(cs, e), size=min(n_rows, e - cs), replace=False))
-            inV, inS = vo.membership(e, V), vo.membership(e, S)
-            # two-point fit: one row (the call's fixed cost, e.g. rotating the keys) and all rows
-            vo.attention_rows(qf[rows[-1:]], rows[-1:], kf, vf, e, inV, inS, w.rope_base, scale, dca)
-            t2 = time.time()
-            vo.attention_rows(qf[rows], rows, kf, vf, e, inV, inS, w.rope_base, scale, dca)
-            t3 = time.time()
-            per_row = max(t3 - t2 - (t2 - t1), 0.0) / max(len(rows) - 1, 1)
-            fixed = max((t2 - t1) - per_row, 0.0)
-            t_fixed += (t1 - t0) + fixed
-            t_rows += per_row * (e - cs)  # extrapolated to every row of the chunk
-            rows_done += len(rows)
-    per_head = (t_fixed + t_rows) / len(heads)
-    layer_s = per_head * w.hq
-    desc = (f"{len(heads)} of {w.hq} heads; per head all {w.n_chunks} chunks' estimation+selection"
-            f"{'+refinement' if w.refine_tau else ''} and {n_rows} sampled query rows per chunk, extrapolated "
-            f"to every row and head")
+        if ("k", hk) not in cache:
+            cache = {k: v for k, v in cache.items() if k[0] != "k" and k[0] != "v"}
+            cache[("k", hk)] = generate_head(w, "k", hk, st=st).float().double().numpy()
+            cache[("v", hk)] = generate_head(w, "v", hk, st=st).float().double().numpy()
+        if ("q", h) not in cache:
+            cache = {k: v for k, v in cache.items() if k[0] != "q"}
+            cache[("q", h)] = generate_head(w, "q", h, st=st).float().double().numpy()
+        kf, vf, qf = cache[("k", hk)], cache[("v", hk)], cache[("q", h)]
+        cs, e = w.chunk_bounds(c)
+        nr = min(w.last_q, e - cs)
+        t0 = time.time()
+        _, vert, slash, a = vo.estimate(qf[e - nr : e], kf, e, w.rope_base, scale)
+        if w.refine_tau is None:
+            V, S = vo.select(vert, slash, w.kv_budget, w.ks_budget)
+        else:
+            _, _, V, S, _, _ = vo.refine(a, np.arange(e - nr, e), vert, slash, w.kv_budget, w.ks_budget,
+                                         w.refine_tau)
+        t1 = time.time()
+        rows = np.sort(rng.choice(np.arange(cs, e), size=min(n_rows, e - cs), replace=False))
+        inV, inS = vo.membership(e, V), vo.membership(e, S)
+        # two-point fit: one row (the call's fixed cost, e.g. rotating the keys) and all rows
+        vo.attention_rows(qf[rows[-1:]], rows[-1:], kf, vf, e, inV, inS, w.rope_base, scale, dca)
+        t2 = time.time()
+        vo.attention_rows(qf[rows], rows, kf, vf, e, inV, inS, w.rope_base, scale, dca)
+        t3 = time.time()
+        per_row = max(t3 - t2 - (t2 - t1), 0.0) / max(len(rows) - 1, 1)
+        fixed = max((t2 - t1) - per_row, 0.0)
+        fixed_per_key.append(((t1 - t0) + fixed) / e)
+        row_per_key.append(per_row / e)
+        done += 1
+    fk, rk = float(np.mean(fixed_per_key)), float(np.mean(row_per_key))
+    layer_s = 0.0
+    for c in range(w.n_chunks):
+        cs, e = w.chunk_bounds(c)
+        layer_s += w.hq * (fk * e + rk * e * (e - cs))
+    desc = (f"{done} of {len(units)} (head, chunk) units, each the chunk's estimation+selection"
+            f"{'+refinement' if w.refine_tau else ''} for one head and {n_rows} sampled query rows of its "
+            f"attention; per-key rates extrapolated to every row, chunk and head")
     return w.seq_len / layer_s, time.time() - spent0, desc
 
 
@@ -436,10 +450,10 @@ def cpu_cores():
 def run_reference(args):
     w = select_workload(args)
     for _ in range(args.warmup):
-        oracle_sample(w, n_heads=1, n_rows=8, seed=99)
+        oracle_sample(w, budget_s=2.0, n_rows=16, seed=99)
     vals = []
     for i in range(args.steps):
-        v, spent, desc = oracle_sample(w, n_heads=1, n_rows=16, seed=i)
+        v, spent, desc = oracle_sample(w, budget_s=8.0, n_rows=32, seed=i)
         vals.append(v)
     value = statistics.median(vals)
     cb = {"value": round(value, 3), "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle", "sample": desc}
@@ -476,8 +490,7 @@ def main():
                                              device_id=device)
     res, w, lay = run_ours(args, rank, world, device)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        n_heads, n_rows = (1, 64)
-        v, spent, desc = oracle_sample(w, n_heads=n_heads, n_rows=n_rows)
+        v, spent, desc = oracle_sample(w, budget_s=15.0, n_rows=64)
         res["cpu_baseline"] = {"value": round(v, 3), "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
                                "sample": desc, "seconds": round(spent, 1)}
     if world > 1:

@@ -20,8 +20,9 @@
 //           index, splitting wrapped / unwrapped parts and transpose-summing
 //           both; written as per-(head, 32-row half) partial arrays that a fixup
 //           kernel adds in a fixed order (deterministic, no atomics)
-//   kRecall A = exp(s - lse) binned by the first refinement level that selects
-//           the element (min of its column's and its offset's level)
+//   kRecall A = exp(s - lse) added to every refinement level that selects the
+//           element: the levels t >= min(its column's level, its offset's level),
+//           so level t accumulates the recall mass of C_t directly
 #include <algorithm>
 #include <cmath>
 
@@ -294,20 +295,27 @@ __global__ void __launch_bounds__(kEstThreads, 1)
               }
             } else {  // kRecall
               if (row_ok) {
+                // acc[t] is cumulative: it gathers A of the elements whose level is <= t.
+                // An element's level set is the bitmask ~0 << lv (levels t >= lv),
+                // restricted to the levels in use; masked-out (j > irow) elements have
+                // v = 0 and read a clamped, in-range offset.
                 const uint8_t* lv_v = p.lvl + static_cast<int64_t>(h) * 2 * p.e_pad;
                 const uint8_t* lv_s = lv_v + p.e_pad;
+                const uint32_t levmask = (1u << p.nlev) - 1u;
+                uint32_t vw[8];  // the 32 columns' vertical levels, 4 per word (same for all lanes)
+#pragma unroll
+                for (int q = 0; q < 8; ++q) vw[q] = __ldg(reinterpret_cast<const uint32_t*>(lv_v + j0) + q);
 #pragma unroll
                 for (int x = 0; x < 32; ++x) {
-                  const int64_t j = j0 + x;
-                  if (j <= irow) {
-                    const int lvv = __ldg(lv_v + j);
-                    const int lvs = __ldg(lv_s + (irow - j));
-                    const int lv = lvv < lvs ? lvv : lvs;
+                  const int64_t d = irow - (j0 + x);
+                  const uint32_t lvv = (vw[x >> 2] >> (8 * (x & 3))) & 0xFFu;
+                  const uint32_t lvs = __ldg(lv_s + (d >= 0 ? d : 0));
+                  const uint32_t lv = lvv < lvs ? lvv : lvs;
+                  const uint32_t lm = lv < 32u ? ((0xFFFFFFFFu << lv) & levmask) : 0u;
 #pragma unroll
-                    for (int t2 = 0; t2 < kRecallLevels; ++t2) {
-                      if (t2 >= p.nlev) break;  // uniform: levels in use only
-                      acc[a][t2] += (lv == t2) ? v[x] : 0.f;
-                    }
+                  for (int t2 = 0; t2 < kRecallLevels; ++t2) {
+                    if (t2 >= p.nlev) break;  // uniform: levels in use only
+                    if ((lm >> t2) & 1u) acc[a][t2] += v[x];
                   }
                 }
               }

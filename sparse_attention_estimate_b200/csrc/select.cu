@@ -257,7 +257,7 @@ __global__ void refine_decide_kernel(const float* __restrict__ hist, int nsplit,
     double m = 0.0;
     for (int s = 0; s < nsplit; ++s)
       m += static_cast<double>(hist[(static_cast<int64_t>(s) * hq + h) * kMaxLevels + t]);
-    cum += m;
+    cum = m;  // the histogram is cumulative: level t holds the recall mass of C_t
     rc = cum / nr;
     kvt = (kv0 << t) > e ? e : (kv0 << t);
     kst = (ks0 << t) > e ? e : (ks0 << t);
