@@ -42,6 +42,26 @@ from workloads import WORKLOADS, generate_head, structure  # noqa: E402
 METRIC = "sparse-prefill tokens/s per layer; executed TFLOP/s and % of B200 BF16 peak"
 FLOP_PER_TILE = 4 * 128 * 128 * 128  # QK^T and PV of one executed 128-query x 128-key tile
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# DRAM bytes (read + write) of one attention-kernel launch, from one ncu capture per
+# workload (profiles/attn_kernel_*.md), valid only for the kernel sources they were
+# taken on: a sha256 prefix over attn.cu, sm100.cuh and internal.cuh. A changed
+# kernel reports null until it is captured again.
+ATTN_TRAFFIC = {
+    "cfg2_qwen7b_n32k_refine": ("84f38628919075ac", 686018816 + 203208448),
+}
+
+
+def attn_traffic(workload: str):
+    import hashlib
+
+    rec = ATTN_TRAFFIC.get(workload)
+    if rec is None:
+        return None
+    h = hashlib.sha256()
+    for f in ("attn.cu", "sm100.cuh", "internal.cuh"):
+        with open(os.path.join(ROOT, "sparse_attention_estimate_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return rec[1] if h.hexdigest().startswith(rec[0]) else None
 
 
 def log(*a):
@@ -325,7 +345,8 @@ def run_ours(args, rank, world, device):
         "roofline": {
             "bound": "tensor", "kernel": "attn_kernel",
             "achieved": round(attn_tflops, 2), "peak": peak, "unit": "TFLOP/s",
-            "frac": round(attn_tflops / peak, 4), "traffic": None,
+            "frac": round(attn_tflops / peak, 4), "traffic": attn_traffic(w.name),
+            "traffic_unit": "DRAM bytes per launch (ncu)",
             "peak_kind": f"{pk_src} {'sustained' if long_step else 'burst'} bf16",
             "flop_per_launch": round(exec_flops / nchunks),
         },
