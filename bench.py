@@ -80,6 +80,9 @@ def parse():
     p.add_argument("--max-iters", type=int, default=19)
     p.add_argument("--seq-len", type=int, default=None,
                    help="prefill only the first SEQ_LEN tokens of the workload (profiling cases)")
+    p.add_argument("--mask", choices=["selected", "full"], default="selected",
+                   help="full: the dense causal baseline through the same attention kernel (every key "
+                        "of [0, e) selected; no estimation or selection)")
     return p.parse_args()
 
 
@@ -184,11 +187,12 @@ class ClockSampler:
 class Layer:
     """One layer's inputs on the device, the library context and per-chunk buffers."""
 
-    def __init__(self, w, device, max_iters):
+    def __init__(self, w, device, max_iters, full_mask=False):
         import sparse_attention_estimate_b200 as vsb
 
         self.vsb = vsb
         self.w = w
+        self.full_mask = full_mask
         self.dev = device
         self.max_iters = max_iters
         st = structure(w)
@@ -204,7 +208,7 @@ class Layer:
         self.lse = torch.empty(w.hq, w.seq_len, dtype=torch.float32, device=device)
         C = w.dca_chunk
         cfg = vsb.Config(hq=w.hq, hkv=w.hkv, rope_base=w.rope_base, last_q=w.last_q, dca_chunk=C,
-                         dca_window=w.dca_window if C else None)
+                         dca_window=w.dca_window if C else None, softmax_scale=w.softmax_scale)
         self.ctx = vsb.Context(cfg, max_seq=w.seq_len, max_chunk=min(w.chunk, w.seq_len), device=device)
         e_max = w.seq_len
         self.vert = torch.empty(w.hq, e_max, dtype=torch.float32, device=device)
@@ -220,6 +224,9 @@ class Layer:
                      torch.empty(w.hq, e_max, dtype=torch.int32, device=device),
                      torch.empty(w.hq, dtype=torch.int32, device=device))
         self.chunks = [w.chunk_bounds(c) for c in range(w.n_chunks)]
+        if full_mask:  # every column of [0, e) is a selected vertical: the dense causal mask
+            self.sets[0].copy_(torch.arange(e_max, dtype=torch.int32, device=device).expand(w.hq, e_max))
+            self.sets[3].zero_()
 
     def step(self, attn_events=None, stats=None, q=None, k=None, v=None):
         """One pass of the whole hot path. attn_events: list of (start, stop) per
@@ -232,6 +239,10 @@ class Layer:
         ctx.reset()  # every step rotates its keys again
         for ci, (cs, e) in enumerate(self.chunks):
             vert, slash = self.vert[:, :e], self.slash[:, :e]
+            if self.full_mask:
+                self.sets[1].fill_(e)
+                self._attend(ci, cs, e, q, k, v, attn_events, stats)
+                continue
             ctx.estimate(q, cs, k, e, out=(self.vert, self.slash, self.lse_est), full=True)
             self.kv.copy_(self.base_v)
             self.ks.copy_(self.base_s)
@@ -240,14 +251,18 @@ class Layer:
             else:
                 ctx.refine(q, cs, k, e, self.vert, self.slash, self.lse_est, w.refine_tau, self.kv, self.ks,
                            max_iters=self.max_iters, sets=self.sets, recall=self.recall, full=True)
-            if attn_events is not None:
-                ctx.set_prefill_events(*attn_events[ci])
-            ctx.sparse_prefill(q, cs, e, k, v, self.sets, out=self.out, lse=self.lse, full=True)
-            if attn_events is not None:
-                ctx.set_prefill_events(None, None)
-            if stats is not None:
-                stats.append(ctx.prefill_stats())
+            self._attend(ci, cs, e, q, k, v, attn_events, stats)
             del vert, slash
+
+    def _attend(self, ci, cs, e, q, k, v, attn_events, stats):
+        ctx = self.ctx
+        if attn_events is not None:
+            ctx.set_prefill_events(*attn_events[ci])
+        ctx.sparse_prefill(q, cs, e, k, v, self.sets, out=self.out, lse=self.lse, full=True)
+        if attn_events is not None:
+            ctx.set_prefill_events(None, None)
+        if stats is not None:
+            stats.append(ctx.prefill_stats())
 
 
 def flush_l2(buf):
@@ -261,7 +276,7 @@ def run_ours(args, rank, world, device):
     vsbuild.build()
     vsb.load_library()
     w = rank_workload(select_workload(args), rank)
-    lay = Layer(w, device, args.max_iters)
+    lay = Layer(w, device, args.max_iters, full_mask=args.mask == "full")
     l2 = torch.empty(256 << 20, dtype=torch.uint8, device=device)  # > 126 MB L2
     nchunks = len(lay.chunks)
 
@@ -327,9 +342,12 @@ def run_ours(args, rank, world, device):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "bf16",
-        "data": "synthetic (seeded generator: N(0,1) Q/K/V, planted verticals, 64-aligned band)",
+        "data": ("synthetic (seeded generator: N(0,1) Q/K/V" + (f", Q's N(0,1) part x{w.q_scale:g}" if w.q_scale != 1
+                 else "") + ", planted verticals, 64-aligned band)"),
         "config": {
-            "workload": w.name, "seq_len": w.seq_len, "hq": w.hq, "hkv": w.hkv, "head_dim": 128,
+            "workload": w.name + ("_fullmask" if args.mask == "full" else ""), "seq_len": w.seq_len,
+            "hq": w.hq, "hkv": w.hkv, "head_dim": 128, "mask": args.mask, "q_scale": w.q_scale,
+            "softmax_scale": round(w.softmax_scale, 6),
             "chunk": w.chunk, "n_chunks": nchunks, "dca": [w.dca_chunk, w.dca_window] if w.dca_chunk else None,
             "budgets": [w.kv_budget, w.ks_budget], "refine_tau": w.refine_tau,
             "parallelism": f"independent layer per GPU x{world}" if world > 1 else "single GPU",
@@ -409,7 +427,7 @@ def oracle_sample(w, budget_s=15.0, n_rows=64, seed=0):
     st = structure(w)
     rng = np.random.default_rng(seed)
     dca = (w.dca_chunk, w.dca_window) if w.dca_chunk else None
-    scale = 1.0 / math.sqrt(w.head_dim)
+    scale = w.softmax_scale
     chunks = list(range(w.n_chunks - 1, -1, -1))
     units = [(h, c) for c in chunks for h in range(w.hq)]
     fixed_per_key, row_per_key = [], []  # seconds per key of e: per chunk, and per row and chunk
@@ -510,7 +528,7 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=device)
     res, w, lay = run_ours(args, rank, world, device)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.mask == "selected":
         v, spent, desc = oracle_sample(w, budget_s=15.0, n_rows=64)
         res["cpu_baseline"] = {"value": round(v, 3), "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
                                "sample": desc, "seconds": round(spent, 1)}

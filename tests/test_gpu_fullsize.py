@@ -1,9 +1,9 @@
-"""Full-size parity: the five workloads at their real sizes, run through the
+"""Full-size parity: the eight workloads at their real sizes, run through the
 same chunk loop the benchmark times, checked against the oracle on sampled
 query rows, on the complete index sets of sampled (chunk, head) pairs, and on
 properties that hold at any size.
 
-Sampling (fixed seeds): workloads 1 and 2 check every head; 3-5 check a fixed
+Sampling (fixed seeds): workloads 1, 2 and 6 check every head; 3-5, 7, 8 check a fixed
 subset of chunks and heads (the oracle's fp64 estimation of one (chunk, head)
 at e = 1M costs seconds). Rows: uniform without replacement from
 numpy default_rng(seed + 1000), sorted, the same rows for every checked head.
@@ -30,6 +30,9 @@ PLAN = {
     3: ([0, 3], [0, 13, 27], 32),
     4: ([0, 3, 7], [0, 21, 39], 32),
     5: ([0, 9, 31], [0, 39], 16),
+    6: (None, None, 64),
+    7: ([0, 31], [0, 39], 16),
+    8: ([31], [0, 17], 16),
 }
 
 
@@ -54,7 +57,7 @@ def _run_gpu(w, check_chunks):
         for h in range(nh):
             t[h].copy_(generate_head(w, name, h, st=st))
     cfg = vsb.Config(hq=w.hq, hkv=w.hkv, rope_base=w.rope_base, last_q=w.last_q, dca_chunk=w.dca_chunk,
-                     dca_window=w.dca_window)
+                     dca_window=w.dca_window, softmax_scale=w.softmax_scale)
     ctx = vsb.Context(cfg, max_seq=w.seq_len, max_chunk=min(w.chunk, w.seq_len))
     out = torch.empty_like(q)
     lse_o = torch.empty(w.hq, w.seq_len, dtype=torch.float32, device=dev)
@@ -80,13 +83,13 @@ def _run_gpu(w, check_chunks):
     return res, out, st
 
 
-@pytest.mark.parametrize("cfg", [1, 2, 3, 4, 5])
+@pytest.mark.parametrize("cfg", sorted(PLAN))
 def test_fullsize_workload(cfg):
     w = WORKLOADS[cfg]
     chunks_sel, heads_sel, nrows = PLAN[cfg]
     chunks = list(range(w.n_chunks)) if chunks_sel is None else chunks_sel
     res, out, st = _run_gpu(w, set(chunks))
-    scale = 1.0 / math.sqrt(w.head_dim)
+    scale = w.softmax_scale
     dca = (w.dca_chunk, w.dca_window) if w.dca_chunk else None
     heads = range(w.hq) if heads_sel is None else heads_sel
     rng = np.random.default_rng(w.seed + 1000)
@@ -139,5 +142,5 @@ def test_fullsize_workload(cfg):
             oo, ol = vo.attention_rows(q_rows, rows, kf, vf, e, vo.membership(e, V[h]), vo.membership(e, S[h]),
                                        w.rope_base, scale, dca)
             got = f64(out[h][torch.as_tensor(rows, device=out.device)])
-            assert_outputs_close(got, oo, f"cfg{cfg} chunk {c} head {h}")
+            assert_outputs_close(got, oo, f"cfg{cfg} chunk {c} head {h}", w=w)
             assert np.allclose(f64(r["lse"][h, rows - cs]), ol, rtol=0, atol=2e-3), (cfg, c, h)

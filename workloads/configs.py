@@ -9,6 +9,7 @@ W = C / 32, stride S = C - W (the reading recorded in the design doc).
 """
 from __future__ import annotations
 
+import math
 from dataclasses import dataclass, replace
 from typing import Optional
 
@@ -29,6 +30,14 @@ class Workload:
     head_dim: int = 128
     rope_base: float = 1.0e7
     last_q: int = 64
+    # Sparse-regime variant: the N(0, 1) part of Q is multiplied by q_scale, so the
+    # base scaled logits q.k / sqrt(D) have standard deviation q_scale (band and
+    # planted columns unchanged).
+    q_scale: float = 1.0
+    # YaRN attention temperature (explainer, "Length Extrapolation"): with
+    # s = max(1, seq_len / yarn_train_len), sqrt(1/t) = 0.1 ln(s) + 1 and the logits
+    # are divided by t sqrt(D). None: t = 1.
+    yarn_train_len: Optional[int] = None
 
     @property
     def dca_window(self) -> Optional[int]:
@@ -37,6 +46,19 @@ class Workload:
     @property
     def dca_stride(self) -> Optional[int]:
         return None if self.dca_chunk is None else self.dca_chunk - self.dca_chunk // 32
+
+    @property
+    def yarn_factor(self) -> float:
+        """1 / t of the YaRN temperature (1.0 without YaRN)."""
+        if self.yarn_train_len is None:
+            return 1.0
+        s = max(1.0, self.seq_len / self.yarn_train_len)
+        return (0.1 * math.log(s) + 1.0) ** 2
+
+    @property
+    def softmax_scale(self) -> float:
+        """The scale of q.k in the softmax: 1 / (t sqrt(D))."""
+        return self.yarn_factor / math.sqrt(self.head_dim)
 
     @property
     def group(self) -> int:
@@ -63,6 +85,16 @@ WORKLOADS: dict[int, Workload] = {
     5: Workload("cfg5_14b_n1m_dca256k_refine", hq=40, hkv=8, seq_len=1048576, seed=4,
                 n_planted=1024, kv_budget=1000, ks_budget=2048, refine_tau=0.9,
                 dca_chunk=262144),
+    # Next rows: the sparse regime (peaked base logits, std 4) of configs 2 and 5, and
+    # config 5 with the YaRN temperature for 1M tokens over a 262,144-token training length.
+    6: Workload("cfg6_qwen7b_n32k_refine_peaked", hq=28, hkv=4, seq_len=32768, seed=1, n_planted=64,
+                kv_budget=1000, ks_budget=2048, refine_tau=0.9, q_scale=4.0),
+    7: Workload("cfg7_14b_n1m_dca256k_refine_peaked", hq=40, hkv=8, seq_len=1048576, seed=4,
+                n_planted=1024, kv_budget=1000, ks_budget=2048, refine_tau=0.9, dca_chunk=262144,
+                q_scale=4.0),
+    8: Workload("cfg8_14b_n1m_dca256k_refine_yarn", hq=40, hkv=8, seq_len=1048576, seed=4,
+                n_planted=1024, kv_budget=1000, ks_budget=2048, refine_tau=0.9, dca_chunk=262144,
+                yarn_train_len=262144),
 }
 
 
@@ -71,6 +103,7 @@ def small_workload(base: int, seq_len: int, chunk: int, *, hq: Optional[int] = N
                    kv_budget: Optional[int] = None, ks_budget: Optional[int] = None,
                    dca_chunk: Optional[int] = None, seed: Optional[int] = None,
                    refine_tau: Optional[float] = -1.0, head_dim: Optional[int] = None,
+                   q_scale: Optional[float] = None, yarn_train_len: Optional[int] = None,
                    name: Optional[str] = None) -> Workload:
     """A reduced copy of workload `base` (same generator recipe, smaller sizes)."""
     w = WORKLOADS[base]
@@ -93,5 +126,9 @@ def small_workload(base: int, seq_len: int, chunk: int, *, hq: Optional[int] = N
         kw["refine_tau"] = refine_tau
     if head_dim is not None:
         kw["head_dim"] = head_dim
+    if q_scale is not None:
+        kw["q_scale"] = q_scale
+    if yarn_train_len is not None:
+        kw["yarn_train_len"] = yarn_train_len
     kw["name"] = name or f"{w.name}_small_n{seq_len}_c{chunk}"
     return replace(w, **kw)

@@ -18,6 +18,8 @@ to bf16):
   adds 2 to the scaled logit of every pair inside an aligned 64 x 64 diagonal
   block.
 * V carries no structure.
+* Sparse-regime variant (q_scale != 1): the N(0, 1) part of Q is multiplied by
+  q_scale before the structure is added, so base scaled logits have std q_scale.
 """
 from __future__ import annotations
 
@@ -88,6 +90,8 @@ def generate_head(w: Workload, tensor: str, head: int, rows: Optional[torch.Tens
     else:
         pos = torch.arange(n)
     if tensor == "q":
+        if w.q_scale != 1.0:
+            x *= w.q_scale  # sparse-regime variant: base logits with std q_scale
         x += 1.5 * st["u"]
         x += _band_amp(d) * st["z"][pos // 64]
     elif tensor == "k":
