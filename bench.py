@@ -20,6 +20,7 @@ workload, extrapolated to the layer.
 from __future__ import annotations
 
 import argparse
+import faulthandler
 import json
 import math
 import os
@@ -43,7 +44,7 @@ METRIC = "sparse-prefill tokens/s per layer; executed TFLOP/s and % of B200 BF16
 FLOP_PER_TILE = 4 * 128 * 128 * 128  # QK^T and PV of one executed 128-query x 128-key tile
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes (read + write) of one attention-kernel launch, from one ncu capture per
-# workload (profiles/attn_kernel_*.md), valid only for the kernel sources they were
+# workload (the attention-kernel summaries under profiles/), valid only for the kernel sources they were
 # taken on: a sha256 prefix over attn.cu, sm100.cuh and internal.cuh. A changed
 # kernel reports null until it is captured again.
 ATTN_TRAFFIC = {
@@ -80,6 +81,9 @@ def parse():
     p.add_argument("--max-iters", type=int, default=19)
     p.add_argument("--seq-len", type=int, default=None,
                    help="prefill only the first SEQ_LEN tokens of the workload (profiling cases)")
+    p.add_argument("--calibrate", action="store_true",
+                   help="offline refinement: per-head budgets calibrated once (outside the timed region) on "
+                        "another sequence of the same workload (seed + 7919); the timed steps select with them")
     p.add_argument("--mask", choices=["selected", "full"], default="selected",
                    help="full: the dense causal baseline through the same attention kernel (every key "
                         "of [0, e) selected; no estimation or selection)")
@@ -122,8 +126,29 @@ def peaks():
 
 
 # ----------------------------------------------------------------------------- clocks
+_NVML_LOOP = r"""
+import sys, time
+import pynvml as nv
+nv.nvmlInit()
+bus, idx = sys.argv[1], int(sys.argv[2])
+h = nv.nvmlDeviceGetHandleByPciBusId(bus) if bus else nv.nvmlDeviceGetHandleByIndex(idx)
+bits = (nv.nvmlClocksEventReasonHwSlowdown, nv.nvmlClocksEventReasonHwThermalSlowdown,
+        nv.nvmlClocksEventReasonSwThermalSlowdown, nv.nvmlClocksEventReasonSwPowerCap)
+mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+print("ready", flush=True)
+while True:
+    sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+    r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+    pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+    print(", ".join([str(sm), str(mx), f"{pw:.1f}"] + ["Active" if r & b else "Not Active" for b in bits]), flush=True)
+    time.sleep(0.005)
+"""
+
+
 class ClockSampler:
-    """Samples SM clock and throttle reasons with nvidia-smi during the timed region."""
+    """Samples the SM clock and the clock-event (throttle) reasons during the timed
+    region, in a child process (read-only queries): NVML every 5 ms when its Python
+    bindings load, else nvidia-smi every 200 ms."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
@@ -133,21 +158,39 @@ class ClockSampler:
         self.idx = device_index
         self.proc = None
         self.lines = []
+        self.source = None
 
     def __enter__(self):
-        try:
-            bus = torch.cuda.get_device_properties(self.idx).pci_bus_id
-            sel = ["--id=" + bus] if bus else ["-i", str(self.idx)]
+        try:  # the device's PCI address, domain:bus:device.function, as NVML and nvidia-smi take it
+            pr = torch.cuda.get_device_properties(self.idx)
+            bus = f"{int(pr.pci_domain_id):08x}:{int(pr.pci_bus_id):02x}:{int(pr.pci_device_id):02x}.0"
         except Exception:
-            sel = ["-i", str(self.idx)]
-        try:
-            self.proc = subprocess.Popen(["nvidia-smi", *sel, "--query-gpu=" + self.FIELDS,
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
+            bus = ""
+        try:  # NVML loop in a child process; it prints "ready" once it samples
+            p = subprocess.Popen([sys.executable, "-c", _NVML_LOOP, bus, str(self.idx)],
+                                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            import select
+
+            ready, _, _ = select.select([p.stdout], [], [], 15.0)
+            first = p.stdout.readline().strip() if ready else ""
+            if first == "ready":
+                self.proc, self.source = p, "nvml, 5 ms"
+            else:
+                p.kill()
         except Exception:
             self.proc = None
+        if self.proc is None:
+            sel = ["--id=" + bus] if bus else ["-i", str(self.idx)]
+            try:
+                self.proc = subprocess.Popen(["nvidia-smi", *sel, "--query-gpu=" + self.FIELDS,
+                                              "--format=csv,noheader,nounits", "-lms", "200"],
+                                             stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                self.source = "nvidia-smi, 200 ms"
+            except Exception:
+                self.proc = None
+        if self.proc is not None:
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
         return self
 
     def _read(self):
@@ -180,7 +223,7 @@ class ClockSampler:
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "source": self.source}
 
 
 # ----------------------------------------------------------------------------- the GPU path
@@ -193,6 +236,7 @@ class Layer:
         self.vsb = vsb
         self.w = w
         self.full_mask = full_mask
+        self.calibrated = False
         self.dev = device
         self.max_iters = max_iters
         st = structure(w)
@@ -224,6 +268,7 @@ class Layer:
                      torch.empty(w.hq, e_max, dtype=torch.int32, device=device),
                      torch.empty(w.hq, dtype=torch.int32, device=device))
         self.chunks = [w.chunk_bounds(c) for c in range(w.n_chunks)]
+        self.cal_summary = None
         if full_mask:  # every column of [0, e) is a selected vertical: the dense causal mask
             self.sets[0].copy_(torch.arange(e_max, dtype=torch.int32, device=device).expand(w.hq, e_max))
             self.sets[3].zero_()
@@ -246,13 +291,39 @@ class Layer:
             ctx.estimate(q, cs, k, e, out=(self.vert, self.slash, self.lse_est), full=True)
             self.kv.copy_(self.base_v)
             self.ks.copy_(self.base_s)
-            if w.refine_tau is None:
+            if w.refine_tau is None or self.calibrated:
                 ctx.select(self.vert, self.slash, e, self.kv, self.ks, sets=self.sets)
             else:
                 ctx.refine(q, cs, k, e, self.vert, self.slash, self.lse_est, w.refine_tau, self.kv, self.ks,
                            max_iters=self.max_iters, sets=self.sets, recall=self.recall, full=True)
             self._attend(ci, cs, e, q, k, v, attn_events, stats)
             del vert, slash
+
+    def calibrate(self):
+        """Per-head budgets from another sequence of the same workload (seed + 7919),
+        generated into the q / k buffers and regenerated afterwards."""
+        w = self.w
+        wc = replace(w, seed=w.seed + 7919)
+        st = structure(wc)
+        for name, t, nh in (("q", self.q, w.hq), ("k", self.k, w.hkv)):
+            for h in range(nh):
+                t[h].copy_(generate_head(wc, name, h, st=st))
+        self.ctx.reset()
+        log(f"[bench] calibrating on {wc.name} seed {wc.seed}")
+        kv, ks = self.vsb.calibrate(self.ctx, self.q, self.k, chunk=w.chunk, kv_budget=w.kv_budget,
+                                    ks_budget=w.ks_budget, tau=w.refine_tau, max_iters=self.max_iters)
+        self.base_v.copy_(kv)
+        self.base_s.copy_(ks)
+        st = structure(w)
+        for name, t, nh in (("q", self.q, w.hq), ("k", self.k, w.hkv)):
+            for h in range(nh):
+                t[h].copy_(generate_head(w, name, h, st=st))
+        self.ctx.reset()
+        self.calibrated = True
+        kvh, ksh = kv.cpu().tolist(), ks.cpu().tolist()
+        self.cal_summary = {"kv": [min(kvh), int(statistics.median(kvh)), max(kvh)],
+                            "ks": [min(ksh), int(statistics.median(ksh)), max(ksh)],
+                            "of": "min / median / max over heads", "sequence": f"seed {wc.seed}"}
 
     def _attend(self, ci, cs, e, q, k, v, attn_events, stats):
         ctx = self.ctx
@@ -277,6 +348,10 @@ def run_ours(args, rank, world, device):
     vsb.load_library()
     w = rank_workload(select_workload(args), rank)
     lay = Layer(w, device, args.max_iters, full_mask=args.mask == "full")
+    if args.calibrate:
+        if w.refine_tau is None or args.mask == "full":
+            raise SystemExit("--calibrate needs a workload with a refinement threshold and --mask selected")
+        lay.calibrate()
     l2 = torch.empty(256 << 20, dtype=torch.uint8, device=device)  # > 126 MB L2
     nchunks = len(lay.chunks)
 
@@ -350,6 +425,7 @@ def run_ours(args, rank, world, device):
             "softmax_scale": round(w.softmax_scale, 6),
             "chunk": w.chunk, "n_chunks": nchunks, "dca": [w.dca_chunk, w.dca_window] if w.dca_chunk else None,
             "budgets": [w.kv_budget, w.ks_budget], "refine_tau": w.refine_tau,
+            "calibrated_budgets": lay.cal_summary,
             "parallelism": f"independent layer per GPU x{world}" if world > 1 else "single GPU",
             "l2": "flushed between steps (256 MiB write)",
         },
@@ -509,6 +585,7 @@ def run_reference(args):
 
 # ----------------------------------------------------------------------------- main
 def main():
+    faulthandler.enable()  # a native crash prints the Python stack to stderr
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

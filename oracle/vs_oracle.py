@@ -24,7 +24,7 @@ dense causal attention; DCA with C >= N equals plain RoPE; DCA's three
 statements on random pairs; RoPE relativity; the recall identity and its
 monotonicity; top-k against a stable lexicographic sort; chunked == unchunked
 under the full mask; MHA and explicit KV repetition for GQA.
-Parity unpinned by the pages (fixed readings): the DCA local
+Parity unpinned by the pages (readings fixed here, none of them stated there): the DCA local
 window W = C/32, doubling both budgets per refinement step, the mean over the
 estimation rows as the head's recall, the forced slash offset 0.
 """
@@ -274,8 +274,33 @@ def attention_rows(q_rows: np.ndarray, rows: np.ndarray, k: np.ndarray, v: np.nd
 
 
 # ----------------------------------------------------------------------------- the chunk loop  [QW Algorithm; Chunked Prefill]
+def calibrate(q: np.ndarray, k: np.ndarray, *, chunk: int, last_q: int, kv_budget: int, ks_budget: int,
+              tau: float, base: float, scale: Optional[float] = None, max_iters: int = 64, heads=None):
+    """Offline form of sparsity refinement ([QW] Chunked Prefill, the sparsity-
+    refinement passage: the budgets are improved once on a calibration sequence).
+    Reading: every chunk of the calibration sequence is refined from the base
+    budgets per head, and a head keeps the largest refined budgets over the chunks
+    (those that reach tau on every chunk). Returns (kv, ks), one int per head."""
+    hq, n, d = q.shape
+    g = hq // k.shape[0]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    heads = list(range(hq)) if heads is None else list(heads)
+    kv_c = {h: 0 for h in heads}
+    ks_c = {h: 0 for h in heads}
+    for cs in range(0, n, chunk):
+        e = min(cs + chunk, n)
+        nr = min(last_q, e - cs)
+        est_rows = np.arange(e - nr, e)
+        for h in heads:
+            _, vert, slash, a = estimate(q[h, e - nr : e], k[h // g], e, base, scale)
+            kv, ks, _, _, _, _ = refine(a, est_rows, vert, slash, kv_budget, ks_budget, tau, max_iters)
+            kv_c[h], ks_c[h] = max(kv_c[h], kv), max(ks_c[h], ks)
+    return [kv_c[h] for h in heads], [ks_c[h] for h in heads]
+
+
 def layer_prefill(q: np.ndarray, k: np.ndarray, v: np.ndarray, *, chunk: int, last_q: int,
-                  kv_budget: int, ks_budget: int, tau: Optional[float], base: float,
+                  kv_budget, ks_budget, tau: Optional[float], base: float,
                   scale: Optional[float] = None, dca: Optional[tuple] = None,
                   rows_per_chunk=None, max_iters: int = 64, heads=None):
     """One attention layer's chunked prefill ([QW] "Algorithm"): for each chunk
@@ -285,6 +310,8 @@ def layer_prefill(q: np.ndarray, k: np.ndarray, v: np.ndarray, *, chunk: int, la
     positions (dca = (C, W)) or continuous ones.
 
     q: (Hq, N, d), k/v: (Hkv, N, d) float64 (bf16 values, pre-RoPE).
+    kv_budget / ks_budget: one int for every head, or a sequence with one budget
+    per head (calibrated budgets, used with tau None).
     rows_per_chunk: None (every row) or a function (cs, e) -> absolute rows to
     evaluate. Returns a list with one dict per chunk."""
     hq, n, d = q.shape
@@ -302,15 +329,16 @@ def layer_prefill(q: np.ndarray, k: np.ndarray, v: np.ndarray, *, chunk: int, la
         per = {}
         for h in heads:
             kh, vh = k[h // g], v[h // g]
+            kvb = int(kv_budget) if np.isscalar(kv_budget) else int(kv_budget[h])
+            ksb = int(ks_budget) if np.isscalar(ks_budget) else int(ks_budget[h])
             lse_e, vert, slash, a = estimate(q[h, e - nr : e], kh, e, base, scale)
             if tau is None:
-                kv, ks = min(kv_budget, e), min(ks_budget, e)
+                kv, ks = min(kvb, e), min(ksb, e)
                 V, S = select(vert, slash, kv, ks)
                 rc = recall(a, est_rows, membership(e, V), membership(e, S))
                 trace = [(kv, ks, rc)]
             else:
-                kv, ks, V, S, rc, trace = refine(a, est_rows, vert, slash, kv_budget, ks_budget, tau,
-                                                 max_iters)
+                kv, ks, V, S, rc, trace = refine(a, est_rows, vert, slash, kvb, ksb, tau, max_iters)
             o, lse = attention_rows(q[h, rows], rows, kh, vh, e, membership(e, V), membership(e, S),
                                     base, scale, dca)
             per[h] = dict(lse_est=lse_e, vert=vert, slash=slash, kv=kv, ks=ks, V=V, S=S,

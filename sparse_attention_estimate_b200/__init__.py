@@ -286,21 +286,48 @@ class Context:
         _check(self.lib.vs_selftest_wait_timeout(self.handle, limit_ns, _stream()))
 
 
+def calibrate(ctx: Context, q: torch.Tensor, k: torch.Tensor, *, chunk: int, kv_budget: int, ks_budget: int,
+              tau: float, max_iters: int = 19):
+    """Offline form of sparsity refinement (explainer, Chunked Prefill: the budgets
+    are improved once on a calibration sequence): every chunk of the calibration
+    sequence q, k is estimated and refined from the base budgets, and each head keeps
+    the largest refined budgets over the chunks. Returns (kv, ks), int32 [hq] on the
+    device, for layer_prefill(..., kv_budget=kv, ks_budget=ks, tau=None)."""
+    hq, n = q.shape[0], q.shape[1]
+    dev = q.device
+    kv_c = torch.zeros(hq, dtype=torch.int32, device=dev)
+    ks_c = torch.zeros(hq, dtype=torch.int32, device=dev)
+    for cs in range(0, n, chunk):
+        e = min(cs + chunk, n)
+        vert, slash, lse = ctx.estimate(q, cs, k, e, full=True)
+        kvb = torch.full((hq,), kv_budget, dtype=torch.int32, device=dev)
+        ksb = torch.full((hq,), ks_budget, dtype=torch.int32, device=dev)
+        ctx.refine(q, cs, k, e, vert, slash, lse, tau, kvb, ksb, max_iters=max_iters, full=True)
+        torch.maximum(kv_c, kvb, out=kv_c)
+        torch.maximum(ks_c, ksb, out=ks_c)
+    return kv_c, ks_c
+
+
 def layer_prefill(ctx: Context, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, chunk: int,
-                  kv_budget: int, ks_budget: int, tau: Optional[float], out: Optional[torch.Tensor] = None,
+                  kv_budget, ks_budget, tau: Optional[float], out: Optional[torch.Tensor] = None,
                   max_iters: int = 19, keep=None):
     """The chunk loop of sparse_attention_with_dca (explainer, "Algorithm"): for
     each chunk [cs, e) of `chunk` queries, estimate with the chunk's last queries,
     select (and refine when tau is given), then attend the chunk's rows over keys
     [0, e). q: [hq, N, 128]; k, v: [hkv, N, 128] (the KV cache, rows at their
-    positions). Returns the output [hq, N, 128] and, when `keep` is a list, appends
-    per-chunk intermediates to it."""
+    positions). kv_budget / ks_budget: ints for every head, or int32 [hq] device
+    tensors (per-head budgets, e.g. from calibrate). Returns the output
+    [hq, N, 128] and, when `keep` is a list, appends per-chunk intermediates to it."""
     hq, n = q.shape[0], q.shape[1]
     dev = q.device
     if out is None:
         out = torch.empty_like(q)
-    base_v = torch.full((hq,), kv_budget, dtype=torch.int32, device=dev)
-    base_s = torch.full((hq,), ks_budget, dtype=torch.int32, device=dev)
+    def per_head(b):
+        if isinstance(b, torch.Tensor):
+            return b.to(device=dev, dtype=torch.int32)
+        return torch.full((hq,), int(b), dtype=torch.int32, device=dev)
+
+    base_v, base_s = per_head(kv_budget), per_head(ks_budget)
     lse_o = torch.empty(hq, n, dtype=torch.float32, device=dev)
     for cs in range(0, n, chunk):
         e = min(cs + chunk, n)

@@ -240,15 +240,10 @@ def test_sparse_prefill_is_deterministic(case):
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
 
 
-def test_layer_prefill_end_to_end(case):
-    """The chunk loop on the GPU against the oracle's chunk loop."""
-    name, w, dca, dev, cpu, ctx = case
-    keep = []
-    out = vsb.layer_prefill(ctx, dev["q"], dev["k"], dev["v"], chunk=w.chunk, kv_budget=w.kv_budget,
-                            ks_budget=w.ks_budget, tau=w.refine_tau, keep=keep)
-    assert ctx.status() == vsb.VS_OK
-    ref = vo.layer_prefill(cpu["q"], cpu["k"], cpu["v"], chunk=w.chunk, last_q=w.last_q, kv_budget=w.kv_budget,
-                           ks_budget=w.ks_budget, tau=w.refine_tau, base=w.rope_base, scale=scale_of(w), dca=dca)
+def _check_layer(name, w, keep, ref, out):
+    """Per chunk and head: identical sets give outputs within tolerance; sets that
+    differ under the same budgets differ only by near-ties; other budgets are only
+    allowed where the oracle's refinement met a recall within TAU_SLACK of tau."""
     out = f64(out)
     for kc, rc in zip(keep, ref):
         V, S = sets_to_lists(kc["sets"])
@@ -267,6 +262,46 @@ def test_layer_prefill_end_to_end(case):
             else:  # other budgets: only a refinement decision at tau may tell them apart
                 assert w.refine_tau is not None and any(
                     abs(x - w.refine_tau) < TAU_SLACK for _, _, x in r["trace"]), (name, rc["cs"], h, r["trace"])
+
+
+def test_layer_prefill_end_to_end(case):
+    """The chunk loop on the GPU against the oracle's chunk loop."""
+    name, w, dca, dev, cpu, ctx = case
+    keep = []
+    out = vsb.layer_prefill(ctx, dev["q"], dev["k"], dev["v"], chunk=w.chunk, kv_budget=w.kv_budget,
+                            ks_budget=w.ks_budget, tau=w.refine_tau, keep=keep)
+    assert ctx.status() == vsb.VS_OK
+    ref = vo.layer_prefill(cpu["q"], cpu["k"], cpu["v"], chunk=w.chunk, last_q=w.last_q, kv_budget=w.kv_budget,
+                           ks_budget=w.ks_budget, tau=w.refine_tau, base=w.rope_base, scale=scale_of(w), dca=dca)
+    _check_layer(name, w, keep, ref, out)
+
+
+def test_calibrated_budgets_and_fixed_budget_prefill(case):
+    """Offline refinement: per-head budgets calibrated on the sequence match the
+    oracle's (up to recalls within TAU_SLACK of tau), and the prefill with those
+    fixed budgets (selection only, no refinement) matches the oracle's."""
+    name, w, dca, dev, cpu, ctx = case
+    if w.refine_tau is None:
+        pytest.skip("no refinement threshold")
+    kv, ks = vsb.calibrate(ctx, dev["q"], dev["k"], chunk=w.chunk, kv_budget=w.kv_budget,
+                           ks_budget=w.ks_budget, tau=w.refine_tau)
+    assert ctx.status() == vsb.VS_OK
+    kw = dict(chunk=w.chunk, last_q=w.last_q, kv_budget=w.kv_budget, ks_budget=w.ks_budget, tau=w.refine_tau,
+              base=w.rope_base, scale=scale_of(w))
+    okv, oks = vo.calibrate(cpu["q"], cpu["k"], **kw)
+    kv_h, ks_h = kv.cpu().numpy(), ks.cpu().numpy()
+    if (list(kv_h), list(ks_h)) != (okv, oks):
+        traces = vo.layer_prefill(cpu["q"], cpu["k"], cpu["v"], **kw, dca=dca, rows_per_chunk=lambda cs, e: [e - 1])
+        for h in range(w.hq):
+            if (kv_h[h], ks_h[h]) != (okv[h], oks[h]):
+                assert any(abs(x - w.refine_tau) < TAU_SLACK for c in traces for _, _, x in c["heads"][h]["trace"])
+    keep = []
+    out = vsb.layer_prefill(ctx, dev["q"], dev["k"], dev["v"], chunk=w.chunk, kv_budget=kv, ks_budget=ks,
+                            tau=None, keep=keep)
+    assert ctx.status() == vsb.VS_OK
+    ref = vo.layer_prefill(cpu["q"], cpu["k"], cpu["v"], **{**kw, "kv_budget": kv_h, "ks_budget": ks_h, "tau": None},
+                           dca=dca)
+    _check_layer(name, w, keep, ref, out)
 
 
 def test_wait_timeout_is_reported_and_context_survives():

@@ -392,6 +392,34 @@ def test_layer_prefill_matches_bruteforce_chain(rng):
         assert np.all(np.abs(r["out"] - np.array(o)) <= 2.0 ** -7 * np.abs(np.array(o)) + 1e-30)
 
 
+def test_calibration_budgets(rng):
+    """Offline refinement: on one chunk the calibrated budgets are the refined ones
+    (brute-force chain); over several chunks each head keeps the largest refined
+    budgets, and with them every chunk's recall reaches tau or both budgets cover
+    the chunk's keys (recall is non-decreasing in the budgets)."""
+    hq, n, d = 2, 72, 8
+    q, k, v = _layer(rng, hq, 1, n, d)
+    scale = 1 / math.sqrt(d)
+    kw = dict(last_q=6, kv_budget=2, ks_budget=1, tau=0.75, base=BASE, scale=scale)
+    kv1, ks1 = vo.calibrate(q[:, :24], k[:, :24], chunk=24, **kw)
+    for h in range(hq):
+        est_q = [list(x) for x in q[h, 18:24]]
+        _, vert, slash, A = bf.estimate(est_q, [list(x) for x in k[0, :24]], 24, BASE, scale)
+        bkv, bks, _, _, _ = bf.refine(A, list(range(18, 24)), vert, slash, 2, 1, 0.75)
+        assert (kv1[h], ks1[h]) == (bkv, bks)
+    kv, ks = vo.calibrate(q, k, chunk=24, **kw)
+    per_chunk = vo.layer_prefill(q, k, v, chunk=24, **{**kw, "tau": 0.75})
+    for h in range(hq):
+        assert kv[h] == max(c["heads"][h]["kv"] for c in per_chunk)
+        assert ks[h] == max(c["heads"][h]["ks"] for c in per_chunk)
+    fixed = vo.layer_prefill(q, k, v, chunk=24, **{**kw, "kv_budget": kv, "ks_budget": ks, "tau": None})
+    for c in fixed:
+        for h in range(hq):
+            r = c["heads"][h]
+            assert r["recall"] >= 0.75 - 1e-12 or (r["kv"] >= c["e"] and r["ks"] >= c["e"])
+            assert r["kv"] == min(kv[h], c["e"]) and r["ks"] == min(ks[h], c["e"])
+
+
 # ------------------------------------------------------------------ sensitivity
 MUTANTS = {
     "rope_sign": lambda x1, x2, c, s: (x1 * c + x2 * s, x2 * c - x1 * s),

@@ -5,7 +5,7 @@ framework" / "Chunked Prefill": 32,768-token chunks, last 64 queries of each
 chunk drive selection; Table 2: final RoPE base 10,000,000) and the two model
 shapes: Qwen2.5-7B (28 query / 4 KV heads, head_dim 128) and a 14B-shaped layer
 (40 / 8). DCA constants: chunk size C as given per workload, local window
-W = C / 32, stride S = C - W (the reading recorded in the design doc).
+W = C / 32, stride S = C - W (a reading: the pages fix C and the three rules only).
 """
 from __future__ import annotations
 
