@@ -12,7 +12,8 @@
 // blocks, and a schedule kernel lists, per CTA, the blocks in which either tile
 // has a selected element, tagging each (tile, block) as skip / partial / full.
 //
-// The attention kernel (one CTA per SM, 12 warps):
+// The attention kernel (one CTA per SM, 12 warps; after the role split the control
+// warpgroup keeps 112 registers per thread and the softmax warpgroups 192):
 //  warp 0     TMA producer: the two Q tiles (re-loaded with another rotation
 //             when the DCA class of the key block changes), K and V blocks into
 //             two-stage rings.
@@ -35,6 +36,11 @@
 namespace vs {
 
 constexpr int kAttnThreads = 384;
+// Register budgets after the role split: warpgroup 0 (TMA producer, MMA issuer, two
+// idle warps) keeps 112 per thread, the two softmax warpgroups take 192 each:
+// 128 x 112 + 256 x 192 = 63488 <= 384 x 168 (the launch's 64512).
+constexpr uint32_t kRegsControl = 112, kRegsSoftmax = 192;
+static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= 384 * 168, "register split exceeds the launch");
 constexpr float kLog2eA = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int kDevErrIndex = 4;            // an index list held an out-of-range entry
@@ -272,162 +278,167 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after_sync();
   const uint32_t tbase = s.tmem_base;
   constexpr uint32_t kTileBytes = kTile * 64 * 2;  // one 128 x 64 bf16 box
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0 && n > 0) {
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-      int cls[2];
-      int qchg[2] = {0, 0};
-      const int64_t kb0 = static_cast<int64_t>(list[0] & 0xFFFFFF) * kTile;
-      for (int t = 0; t < 2; ++t) {
-        cls[t] = dca_class(R0 + t * kTile, kb0, p.dca);
-        mbar_arrive_expect_tx(&s.q_full[t], 2 * kTileBytes);
-        const int qrow = pair * 256 + t * kTile;
-        const int qh = cls[t] * p.hq + h;
-        tma_load_3d(s.q[t][0], &tmQ, &s.q_full[t], 0, qrow, qh);
-        tma_load_3d(s.q[t][1], &tmQ, &s.q_full[t], 64, qrow, qh);
-      }
-      int kiss[2] = {0, 0}, viss[2] = {0, 0};
-      bool ok = true;
-      int32_t ent = list[0];  // schedule entries are read one block ahead of use
-      for (int j = 0; j < n && ok; ++j) {
-        const int b = ent & 0xFFFFFF;
-        ent = j + 1 < n ? ld_keep_s32(list + j + 1) : 0;
-        const int st = j & 1;
-        // K(j) first: the MMA warp releases a Q tile only after issuing S0(j)
-        if (j >= 2) ok = mbar_wait(&s.k_empty[st], ((j >> 1) - 1) & 1, abort_word, p.dc.err);
-        if (!ok) break;
-        mbar_arrive_expect_tx(&s.k_full[st], 2 * kTileBytes);
-        tma_load_3d(s.k[st][0], &tmK, &s.k_full[st], 0, b * kTile, hk);
-        tma_load_3d(s.k[st][1], &tmK, &s.k_full[st], 64, b * kTile, hk);
-        ++kiss[st];
-        if (j > 0) {
-          for (int t = 0; t < 2 && ok; ++t) {
-            const int c = dca_class(R0 + t * kTile, static_cast<int64_t>(b) * kTile, p.dca);
-            if (c != cls[t]) {
-              ok = mbar_wait(&s.q_empty[t], qchg[t] & 1, abort_word, p.dc.err);
-              if (!ok) break;
-              ++qchg[t];
-              cls[t] = c;
-              mbar_arrive_expect_tx(&s.q_full[t], 2 * kTileBytes);
-              const int qrow = pair * 256 + t * kTile;
-              tma_load_3d(s.q[t][0], &tmQ, &s.q_full[t], 0, qrow, c * p.hq + h);
-              tma_load_3d(s.q[t][1], &tmQ, &s.q_full[t], 64, qrow, c * p.hq + h);
-            }
-          }
-          if (!ok) break;
-        }
-        if (j >= 2) ok = mbar_wait(&s.v_empty[st], ((j >> 1) - 1) & 1, abort_word, p.dc.err);
-        if (!ok) break;
-        mbar_arrive_expect_tx(&s.v_full[st], 2 * kTileBytes);
-        tma_load_3d(s.v[st][0], &tmV, &s.v_full[st], 0, b * kTile, hk);
-        tma_load_3d(s.v[st][1], &tmV, &s.v_full[st], 64, b * kTile, hk);
-        ++viss[st];
-      }
-      if (!ok) {  // let every issued copy land before the CTA exits
-        for (int t = 0; t < 2; ++t) drain_wait_a(&s.q_full[t], qchg[t] & 1, p.dc.wait_ns);
-        for (int st = 0; st < 2; ++st) {
-          if (kiss[st] > 0) drain_wait_a(&s.k_full[st], (kiss[st] - 1) & 1, p.dc.wait_ns);
-          if (viss[st] > 0) drain_wait_a(&s.v_full[st], (viss[st] - 1) & 1, p.dc.wait_ns);
-        }
-      }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      if (n > 0) {
-        const uint32_t id_qk = idesc_bf16_f32(128, 128, 0, 0);
-        const uint32_t id_pv = idesc_bf16_f32(128, 128, 0, 1);
-        const uint32_t tS[2] = {tbase, tbase + 128};
-        const uint32_t tO[2] = {tbase + 256, tbase + 384};
-        int cls[2], qph[2] = {1, 1};
+  if (warp < 4) {
+    // warpgroup 0: the TMA producer (warp 0), the MMA issuer (warp 1), two idle warps
+    setmaxnreg_dec<kRegsControl>();
+    if (warp == 0) {
+      // ------------------------------------------------------------ TMA producer
+      if (lane == 0 && n > 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+        int cls[2];
+        int qchg[2] = {0, 0};
         const int64_t kb0 = static_cast<int64_t>(list[0] & 0xFFFFFF) * kTile;
-        cls[0] = dca_class(R0, kb0, p.dca);
-        cls[1] = dca_class(R0 + kTile, kb0, p.dca);
-        int32_t ent1 = n > 1 ? list[1] : 0;  // entry of block j + 1, read a block ahead
-        auto issue_qk = [&](int t, int st) {
-          const uint32_t qa = smem_u32(&s.q[t][0][0]);
-          const uint32_t ka = smem_u32(&s.k[st][0][0]);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * kTileBytes + (kk & 3) * 32;
-            mma_bf16_ss(tS[t], smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024),
-                        id_qk, kk > 0 ? 1u : 0u);
-          }
-        };
-        auto issue_pv = [&](int t, int st, uint32_t acc) {
-          const uint32_t va = smem_u32(&s.v[st][0][0]);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_bf16_ts(tO[t], tS[t] + kk * 8, smem_desc_sw128(va + kk * 2048, kTileBytes, 1024), id_pv,
-                        (acc || kk > 0) ? 1u : 0u);
-        };
-        bool ok = mbar_wait(&s.q_full[0], 0, abort_word, p.dc.err) &&
-                  mbar_wait(&s.q_full[1], 0, abort_word, p.dc.err) &&
-                  mbar_wait(&s.k_full[0], 0, abort_word, p.dc.err);
-        if (ok) {
-          tc_fence_after_sync();
-          issue_qk(0, 0);
-          mma_commit(&s.s_full[0]);
-          issue_qk(1, 0);
-          mma_commit(&s.s_full[1]);
-          mma_commit(&s.k_empty[0]);
+        for (int t = 0; t < 2; ++t) {
+          cls[t] = dca_class(R0 + t * kTile, kb0, p.dca);
+          mbar_arrive_expect_tx(&s.q_full[t], 2 * kTileBytes);
+          const int qrow = pair * 256 + t * kTile;
+          const int qh = cls[t] * p.hq + h;
+          tma_load_3d(s.q[t][0], &tmQ, &s.q_full[t], 0, qrow, qh);
+          tma_load_3d(s.q[t][1], &tmQ, &s.q_full[t], 64, qrow, qh);
         }
+        int kiss[2] = {0, 0}, viss[2] = {0, 0};
+        bool ok = true;
+        int32_t ent = list[0];  // schedule entries are read one block ahead of use
         for (int j = 0; j < n && ok; ++j) {
+          const int b = ent & 0xFFFFFF;
+          ent = j + 1 < n ? ld_keep_s32(list + j + 1) : 0;
           const int st = j & 1;
-          const bool more = j + 1 < n;
-          const int st1 = (j + 1) & 1;
-          const int64_t kb1 = more ? static_cast<int64_t>(ent1 & 0xFFFFFF) * kTile : 0;
-          ent1 = j + 2 < n ? ld_keep_s32(list + j + 2) : 0;
-          // tile 0
-          ok = mbar_wait(&s.p_full[0], j & 1, abort_word, p.dc.err) &&
-               mbar_wait(&s.v_full[st], (j >> 1) & 1, abort_word, p.dc.err);
+          // K(j) first: the MMA warp releases a Q tile only after issuing S0(j)
+          if (j >= 2) ok = mbar_wait(&s.k_empty[st], ((j >> 1) - 1) & 1, abort_word, p.dc.err);
           if (!ok) break;
-          tc_fence_after_sync();
-          issue_pv(0, st, j > 0);
-          if (more) {
-            const int c = dca_class(R0, kb1, p.dca);
-            if (c != cls[0]) {
-              mma_commit(&s.q_empty[0]);
-              ok = mbar_wait(&s.q_full[0], qph[0] & 1, abort_word, p.dc.err);
-              ++qph[0];
-              cls[0] = c;
+          mbar_arrive_expect_tx(&s.k_full[st], 2 * kTileBytes);
+          tma_load_3d(s.k[st][0], &tmK, &s.k_full[st], 0, b * kTile, hk);
+          tma_load_3d(s.k[st][1], &tmK, &s.k_full[st], 64, b * kTile, hk);
+          ++kiss[st];
+          if (j > 0) {
+            for (int t = 0; t < 2 && ok; ++t) {
+              const int c = dca_class(R0 + t * kTile, static_cast<int64_t>(b) * kTile, p.dca);
+              if (c != cls[t]) {
+                ok = mbar_wait(&s.q_empty[t], qchg[t] & 1, abort_word, p.dc.err);
+                if (!ok) break;
+                ++qchg[t];
+                cls[t] = c;
+                mbar_arrive_expect_tx(&s.q_full[t], 2 * kTileBytes);
+                const int qrow = pair * 256 + t * kTile;
+                tma_load_3d(s.q[t][0], &tmQ, &s.q_full[t], 0, qrow, c * p.hq + h);
+                tma_load_3d(s.q[t][1], &tmQ, &s.q_full[t], 64, qrow, c * p.hq + h);
+              }
             }
-            ok = ok && mbar_wait(&s.k_full[st1], ((j + 1) >> 1) & 1, abort_word, p.dc.err);
             if (!ok) break;
-            tc_fence_after_sync();
-            issue_qk(0, st1);
-            mma_commit(&s.s_full[0]);
           }
-          // tile 1
-          ok = mbar_wait(&s.p_full[1], j & 1, abort_word, p.dc.err);
+          if (j >= 2) ok = mbar_wait(&s.v_empty[st], ((j >> 1) - 1) & 1, abort_word, p.dc.err);
           if (!ok) break;
-          tc_fence_after_sync();
-          issue_pv(1, st, j > 0);
-          mma_commit(&s.v_empty[st]);
-          if (more) {
-            const int c = dca_class(R0 + kTile, kb1, p.dca);
-            if (c != cls[1]) {
-              mma_commit(&s.q_empty[1]);
-              ok = mbar_wait(&s.q_full[1], qph[1] & 1, abort_word, p.dc.err);
-              ++qph[1];
-              cls[1] = c;
-            }
-            if (!ok) break;
-            tc_fence_after_sync();
-            issue_qk(1, st1);
-            mma_commit(&s.s_full[1]);
-            mma_commit(&s.k_empty[st1]);
+          mbar_arrive_expect_tx(&s.v_full[st], 2 * kTileBytes);
+          tma_load_3d(s.v[st][0], &tmV, &s.v_full[st], 0, b * kTile, hk);
+          tma_load_3d(s.v[st][1], &tmV, &s.v_full[st], 64, b * kTile, hk);
+          ++viss[st];
+        }
+        if (!ok) {  // let every issued copy land before the CTA exits
+          for (int t = 0; t < 2; ++t) drain_wait_a(&s.q_full[t], qchg[t] & 1, p.dc.wait_ns);
+          for (int st = 0; st < 2; ++st) {
+            if (kiss[st] > 0) drain_wait_a(&s.k_full[st], (kiss[st] - 1) & 1, p.dc.wait_ns);
+            if (viss[st] > 0) drain_wait_a(&s.v_full[st], (viss[st] - 1) & 1, p.dc.wait_ns);
           }
         }
-        mma_commit(&s.drain);
-        drain_wait_a(&s.drain, 0, p.dc.wait_ns);
       }
-      mbar_arrive(&s.o_final);
+    } else if (warp == 1) {
+      // ------------------------------------------------------------ MMA issuer
+      if (lane == 0) {
+        if (n > 0) {
+          const uint32_t id_qk = idesc_bf16_f32(128, 128, 0, 0);
+          const uint32_t id_pv = idesc_bf16_f32(128, 128, 0, 1);
+          const uint32_t tS[2] = {tbase, tbase + 128};
+          const uint32_t tO[2] = {tbase + 256, tbase + 384};
+          int cls[2], qph[2] = {1, 1};
+          const int64_t kb0 = static_cast<int64_t>(list[0] & 0xFFFFFF) * kTile;
+          cls[0] = dca_class(R0, kb0, p.dca);
+          cls[1] = dca_class(R0 + kTile, kb0, p.dca);
+          int32_t ent1 = n > 1 ? list[1] : 0;  // entry of block j + 1, read a block ahead
+          auto issue_qk = [&](int t, int st) {
+            const uint32_t qa = smem_u32(&s.q[t][0][0]);
+            const uint32_t ka = smem_u32(&s.k[st][0][0]);
+  #pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t off = (kk >> 2) * kTileBytes + (kk & 3) * 32;
+              mma_bf16_ss(tS[t], smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024),
+                          id_qk, kk > 0 ? 1u : 0u);
+            }
+          };
+          auto issue_pv = [&](int t, int st, uint32_t acc) {
+            const uint32_t va = smem_u32(&s.v[st][0][0]);
+  #pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma_bf16_ts(tO[t], tS[t] + kk * 8, smem_desc_sw128(va + kk * 2048, kTileBytes, 1024), id_pv,
+                          (acc || kk > 0) ? 1u : 0u);
+          };
+          bool ok = mbar_wait(&s.q_full[0], 0, abort_word, p.dc.err) &&
+                    mbar_wait(&s.q_full[1], 0, abort_word, p.dc.err) &&
+                    mbar_wait(&s.k_full[0], 0, abort_word, p.dc.err);
+          if (ok) {
+            tc_fence_after_sync();
+            issue_qk(0, 0);
+            mma_commit(&s.s_full[0]);
+            issue_qk(1, 0);
+            mma_commit(&s.s_full[1]);
+            mma_commit(&s.k_empty[0]);
+          }
+          for (int j = 0; j < n && ok; ++j) {
+            const int st = j & 1;
+            const bool more = j + 1 < n;
+            const int st1 = (j + 1) & 1;
+            const int64_t kb1 = more ? static_cast<int64_t>(ent1 & 0xFFFFFF) * kTile : 0;
+            ent1 = j + 2 < n ? ld_keep_s32(list + j + 2) : 0;
+            // tile 0
+            ok = mbar_wait(&s.p_full[0], j & 1, abort_word, p.dc.err) &&
+                 mbar_wait(&s.v_full[st], (j >> 1) & 1, abort_word, p.dc.err);
+            if (!ok) break;
+            tc_fence_after_sync();
+            issue_pv(0, st, j > 0);
+            if (more) {
+              const int c = dca_class(R0, kb1, p.dca);
+              if (c != cls[0]) {
+                mma_commit(&s.q_empty[0]);
+                ok = mbar_wait(&s.q_full[0], qph[0] & 1, abort_word, p.dc.err);
+                ++qph[0];
+                cls[0] = c;
+              }
+              ok = ok && mbar_wait(&s.k_full[st1], ((j + 1) >> 1) & 1, abort_word, p.dc.err);
+              if (!ok) break;
+              tc_fence_after_sync();
+              issue_qk(0, st1);
+              mma_commit(&s.s_full[0]);
+            }
+            // tile 1
+            ok = mbar_wait(&s.p_full[1], j & 1, abort_word, p.dc.err);
+            if (!ok) break;
+            tc_fence_after_sync();
+            issue_pv(1, st, j > 0);
+            mma_commit(&s.v_empty[st]);
+            if (more) {
+              const int c = dca_class(R0 + kTile, kb1, p.dca);
+              if (c != cls[1]) {
+                mma_commit(&s.q_empty[1]);
+                ok = mbar_wait(&s.q_full[1], qph[1] & 1, abort_word, p.dc.err);
+                ++qph[1];
+                cls[1] = c;
+              }
+              if (!ok) break;
+              tc_fence_after_sync();
+              issue_qk(1, st1);
+              mma_commit(&s.s_full[1]);
+              mma_commit(&s.k_empty[st1]);
+            }
+          }
+          mma_commit(&s.drain);
+          drain_wait_a(&s.drain, 0, p.dc.wait_ns);
+        }
+        mbar_arrive(&s.o_final);
+      }
     }
-  } else if (warp >= 4) {
+  } else {
+    setmaxnreg_inc<kRegsSoftmax>();
     // ------------------------------------------------------------ softmax warpgroups
     const int t = (warp - 4) >> 2;
     const int wl = warp & 3;
