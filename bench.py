@@ -84,6 +84,9 @@ def parse():
     p.add_argument("--calibrate", action="store_true",
                    help="offline refinement: per-head budgets calibrated once (outside the timed region) on "
                         "another sequence of the same workload (seed + 7919); the timed steps select with them")
+    p.add_argument("--shard", choices=["layers", "heads"], default="layers",
+                   help="N > 1: layers = an independent layer per rank (weak scaling); heads = one layer's "
+                        "KV groups split over the ranks (strong scaling)")
     p.add_argument("--mask", choices=["selected", "full"], default="selected",
                    help="full: the dense causal baseline through the same attention kernel (every key "
                         "of [0, e) selected; no estimation or selection)")
@@ -100,6 +103,19 @@ def select_workload(args):
 def rank_workload(w, rank: int):
     """Rank r > 0 prefills an independent layer: same shapes, seed offset by 1000 r."""
     return w if rank == 0 else replace(w, seed=w.seed + 1000 * rank)
+
+
+def shard_heads(w, rank: int, world: int):
+    """KV-group sharding of one layer (no data crosses KV groups on the path): rank r
+    takes KV heads [r G, (r + 1) G) with G = hkv / world, and their query heads.
+    Returns the rank's workload (same seed, local head counts) and the global index
+    of its first query head and first KV head; the per-head generators make the
+    rank's heads bit-identical to the same heads of the whole layer."""
+    if w.hkv % world:
+        raise ValueError(f"{w.hkv} KV heads do not split over {world} ranks")
+    gk = w.hkv // world
+    local = replace(w, hq=w.group * gk, hkv=gk, name=f"{w.name}_kvshard{rank}of{world}")
+    return local, rank * w.group * gk, rank * gk
 
 
 def max_over_ranks(x: float, world: int, device) -> float:
@@ -230,7 +246,7 @@ class ClockSampler:
 class Layer:
     """One layer's inputs on the device, the library context and per-chunk buffers."""
 
-    def __init__(self, w, device, max_iters, full_mask=False):
+    def __init__(self, w, device, max_iters, full_mask=False, q0=0, k0=0):
         import sparse_attention_estimate_b200 as vsb
 
         self.vsb = vsb
@@ -244,9 +260,10 @@ class Layer:
         self.q = torch.empty(w.hq, w.seq_len, 128, dtype=torch.bfloat16, device=device)
         self.k = torch.empty(w.hkv, w.seq_len, 128, dtype=torch.bfloat16, device=device)
         self.v = torch.empty(w.hkv, w.seq_len, 128, dtype=torch.bfloat16, device=device)
+        self.h0 = {"q": q0, "k": k0, "v": k0}  # global index of the first local head
         for name, t, nh in (("q", self.q, w.hq), ("k", self.k, w.hkv), ("v", self.v, w.hkv)):
             for h in range(nh):
-                t[h].copy_(generate_head(w, name, h, st=st))
+                t[h].copy_(generate_head(w, name, self.h0[name] + h, st=st))
         log(f"[bench] generated {w.name} in {time.time() - t0:.1f}s")
         self.out = torch.empty_like(self.q)
         self.lse = torch.empty(w.hq, w.seq_len, dtype=torch.float32, device=device)
@@ -307,7 +324,7 @@ class Layer:
         st = structure(wc)
         for name, t, nh in (("q", self.q, w.hq), ("k", self.k, w.hkv)):
             for h in range(nh):
-                t[h].copy_(generate_head(wc, name, h, st=st))
+                t[h].copy_(generate_head(wc, name, self.h0[name] + h, st=st))
         self.ctx.reset()
         log(f"[bench] calibrating on {wc.name} seed {wc.seed}")
         kv, ks = self.vsb.calibrate(self.ctx, self.q, self.k, chunk=w.chunk, kv_budget=w.kv_budget,
@@ -317,7 +334,7 @@ class Layer:
         st = structure(w)
         for name, t, nh in (("q", self.q, w.hq), ("k", self.k, w.hkv)):
             for h in range(nh):
-                t[h].copy_(generate_head(w, name, h, st=st))
+                t[h].copy_(generate_head(w, name, self.h0[name] + h, st=st))
         self.ctx.reset()
         self.calibrated = True
         kvh, ksh = kv.cpu().tolist(), ks.cpu().tolist()
@@ -346,8 +363,16 @@ def run_ours(args, rank, world, device):
 
     vsbuild.build()
     vsb.load_library()
-    w = rank_workload(select_workload(args), rank)
-    lay = Layer(w, device, args.max_iters, full_mask=args.mask == "full")
+    if args.shard == "heads" and world > 1:  # one layer, KV groups over the ranks
+        w, q0, k0 = shard_heads(select_workload(args), rank, world)
+        lay = Layer(w, device, args.max_iters, full_mask=args.mask == "full", q0=q0, k0=k0)
+        lay.job_layers = 1
+        wj = select_workload(args)
+    else:  # an independent layer per rank
+        w = rank_workload(select_workload(args), rank)
+        lay = Layer(w, device, args.max_iters, full_mask=args.mask == "full")
+        lay.job_layers = world
+        wj = w
     if args.calibrate:
         if w.refine_tau is None or args.mask == "full":
             raise SystemExit("--calibrate needs a workload with a refinement threshold and --mask selected")
@@ -397,7 +422,7 @@ def run_ours(args, rank, world, device):
     attn_ms = [sum(a.elapsed_time(b) for a, b in evs) for evs in attn_ev]
     tot_ms = max_over_ranks(sum(step_ms), world, device)
     ms_per_step = tot_ms / args.steps
-    value = job_throughput(w.seq_len, args.steps, world, tot_ms)
+    value = job_throughput(w.seq_len, args.steps, lay.job_layers, tot_ms)
     attn_ms_step = sum(attn_ms) / args.steps
     exec_flops = executed * FLOP_PER_TILE
     useful_flops = useful * 4 * 128
@@ -414,19 +439,20 @@ def run_ours(args, rank, world, device):
         "warmup": args.warmup,
         "ms_per_step": round(ms_per_step, 3),
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": "strong" if lay.job_layers == 1 and world > 1 else "weak",
         "vs_baseline": None,
         "dtype": "bf16",
         "data": ("synthetic (seeded generator: N(0,1) Q/K/V" + (f", Q's N(0,1) part x{w.q_scale:g}" if w.q_scale != 1
                  else "") + ", planted verticals, 64-aligned band)"),
         "config": {
-            "workload": w.name + ("_fullmask" if args.mask == "full" else ""), "seq_len": w.seq_len,
-            "hq": w.hq, "hkv": w.hkv, "head_dim": 128, "mask": args.mask, "q_scale": w.q_scale,
+            "workload": wj.name + ("_fullmask" if args.mask == "full" else ""), "seq_len": w.seq_len,
+            "hq": wj.hq, "hkv": wj.hkv, "head_dim": 128, "mask": args.mask, "q_scale": w.q_scale,
             "softmax_scale": round(w.softmax_scale, 6),
             "chunk": w.chunk, "n_chunks": nchunks, "dca": [w.dca_chunk, w.dca_window] if w.dca_chunk else None,
             "budgets": [w.kv_budget, w.ks_budget], "refine_tau": w.refine_tau,
             "calibrated_budgets": lay.cal_summary,
-            "parallelism": f"independent layer per GPU x{world}" if world > 1 else "single GPU",
+            "parallelism": ("single GPU" if world == 1 else f"KV groups of one layer over {world} GPUs"
+                            if lay.job_layers == 1 else f"independent layer per GPU x{world}"),
             "l2": "flushed between steps (256 MiB write)",
         },
         "executed_tflops": round(exec_flops / (ms_per_step / 1e3) / 1e12, 2),
@@ -484,7 +510,7 @@ def run_e2e(args, lay, l2, world, device):
     tot = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), world, device)
     h2d = (hq_h.numel() + hk_h.numel() + hv_h.numel()) * 2
     d2h = out_h.numel() * 2
-    return {"value": round(job_throughput(lay.w.seq_len, args.steps, world, tot), 1), "unit": "tokens/s",
+    return {"value": round(job_throughput(lay.w.seq_len, args.steps, lay.job_layers, tot), 1), "unit": "tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(tot / args.steps, 3)}
 
 

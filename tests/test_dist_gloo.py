@@ -58,3 +58,56 @@ def test_bench_rank_logic_on_two_gloo_ranks():
     assert all(r[3] == 20.0 for r in res)  # max over ranks, seen by every rank
     assert all(abs(r[4] - 32768 * 5 * 2 / 0.020) < 1e-6 for r in res)
     assert all(r[5] for r in res)  # ranks hold different data
+
+
+def _shard_main(rank, world, port, q):
+    import datetime
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        import bench
+        from workloads import generate_head, small_workload, structure
+
+        w = small_workload(2, seq_len=256, chunk=256, hq=8, hkv=4)
+        local, q0, k0 = bench.shard_heads(w, rank, world)
+        st = structure(local)
+        qs = torch.stack([generate_head(local, "q", q0 + h, st=st) for h in range(local.hq)])
+        ks = torch.stack([generate_head(local, "k", k0 + h, st=st) for h in range(local.hkv)])
+        gq = [torch.empty_like(qs) for _ in range(world)]
+        gk = [torch.empty_like(ks) for _ in range(world)]
+        dist.all_gather(gq, qs)
+        dist.all_gather(gk, ks)
+        t_max = bench.max_over_ranks(10.0 * (rank + 1), world, torch.device("cpu"))
+        # plain bytes through the queue (tensors would travel as shared memory that
+        # disappears with the child process)
+        q.put((rank, local.hq, local.hkv, q0, k0, torch.cat(gq).view(torch.int16).numpy().tobytes(),
+               torch.cat(gk).view(torch.int16).numpy().tobytes(), t_max, bench.job_throughput(w.seq_len, 5, 1, t_max)))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.timeout(180)
+def test_kv_group_sharding_on_two_gloo_ranks():
+    """KV-group sharding of one layer: the ranks' heads are disjoint, keep each query
+    head with its KV head, and together are bit-identical to the unsharded layer;
+    the job counts one layer's tokens over the slowest rank's time."""
+    from workloads import generate_layer, small_workload
+
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_shard_main, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=150) for _ in range(world))  # drain before joining: large items
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [(r[1], r[2], r[3], r[4]) for r in res] == [(4, 2, 0, 0), (4, 2, 4, 2)]
+    full = generate_layer(small_workload(2, seq_len=256, chunk=256, hq=8, hkv=4), with_v=False)
+    for r in res:
+        assert r[5] == full["q"].view(torch.int16).numpy().tobytes()
+        assert r[6] == full["k"].view(torch.int16).numpy().tobytes()
+        assert r[7] == 20.0 and abs(r[8] - 256 * 5 / 0.020) < 1e-6
