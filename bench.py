@@ -84,6 +84,9 @@ def parse():
     p.add_argument("--calibrate", action="store_true",
                    help="offline refinement: per-head budgets calibrated once (outside the timed region) on "
                         "another sequence of the same workload (seed + 7919); the timed steps select with them")
+    p.add_argument("--refine-positions", choices=["continuous", "dca"], default="continuous",
+                   help="dca: refinement's recall from the estimation rows' attention at DCA positions "
+                        "(DCA workloads)")
     p.add_argument("--shard", choices=["layers", "heads"], default="layers",
                    help="N > 1: layers = an independent layer per rank (weak scaling); heads = one layer's "
                         "KV groups split over the ranks (strong scaling)")
@@ -246,7 +249,7 @@ class ClockSampler:
 class Layer:
     """One layer's inputs on the device, the library context and per-chunk buffers."""
 
-    def __init__(self, w, device, max_iters, full_mask=False, q0=0, k0=0):
+    def __init__(self, w, device, max_iters, full_mask=False, q0=0, k0=0, refine_dca=False):
         import sparse_attention_estimate_b200 as vsb
 
         self.vsb = vsb
@@ -269,7 +272,8 @@ class Layer:
         self.lse = torch.empty(w.hq, w.seq_len, dtype=torch.float32, device=device)
         C = w.dca_chunk
         cfg = vsb.Config(hq=w.hq, hkv=w.hkv, rope_base=w.rope_base, last_q=w.last_q, dca_chunk=C,
-                         dca_window=w.dca_window if C else None, softmax_scale=w.softmax_scale)
+                         dca_window=w.dca_window if C else None, softmax_scale=w.softmax_scale,
+                         refine_dca_positions=refine_dca)
         self.ctx = vsb.Context(cfg, max_seq=w.seq_len, max_chunk=min(w.chunk, w.seq_len), device=device)
         e_max = w.seq_len
         self.vert = torch.empty(w.hq, e_max, dtype=torch.float32, device=device)
@@ -365,12 +369,14 @@ def run_ours(args, rank, world, device):
     vsb.load_library()
     if args.shard == "heads" and world > 1:  # one layer, KV groups over the ranks
         w, q0, k0 = shard_heads(select_workload(args), rank, world)
-        lay = Layer(w, device, args.max_iters, full_mask=args.mask == "full", q0=q0, k0=k0)
+        lay = Layer(w, device, args.max_iters, full_mask=args.mask == "full", q0=q0, k0=k0,
+                    refine_dca=args.refine_positions == "dca")
         lay.job_layers = 1
         wj = select_workload(args)
     else:  # an independent layer per rank
         w = rank_workload(select_workload(args), rank)
-        lay = Layer(w, device, args.max_iters, full_mask=args.mask == "full")
+        lay = Layer(w, device, args.max_iters, full_mask=args.mask == "full",
+                    refine_dca=args.refine_positions == "dca")
         lay.job_layers = world
         wj = w
     if args.calibrate:
@@ -450,7 +456,7 @@ def run_ours(args, rank, world, device):
             "softmax_scale": round(w.softmax_scale, 6),
             "chunk": w.chunk, "n_chunks": nchunks, "dca": [w.dca_chunk, w.dca_window] if w.dca_chunk else None,
             "budgets": [w.kv_budget, w.ks_budget], "refine_tau": w.refine_tau,
-            "calibrated_budgets": lay.cal_summary,
+            "calibrated_budgets": lay.cal_summary, "refine_positions": args.refine_positions,
             "parallelism": ("single GPU" if world == 1 else f"KV groups of one layer over {world} GPUs"
                             if lay.job_layers == 1 else f"independent layer per GPU x{world}"),
             "l2": "flushed between steps (256 MiB write)",

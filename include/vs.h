@@ -69,6 +69,11 @@ typedef struct {
   int32_t dca_enabled;     /* 0: continuous positions in attention; 1: DCA positions */
   int64_t dca_chunk_size;  /* DCA chunk size C (the largest relative position is C-1) */
   int64_t dca_local_window;/* DCA local window W, 0 <= W < C; chunk stride S = C - W */
+  int32_t refine_dca_positions; /* 0: vs_refine measures recall with continuous positions
+                           (the pages' selection positions); 1 (DCA enabled only): recall from
+                           the estimation rows' attention at DCA positions, the attention the
+                           prefill computes. Needs S % 128 == 0 and the estimation rows inside
+                           one DCA chunk, else vs_refine returns VS_ERR_UNSUPPORTED. */
 } vs_attn_cfg;
 
 typedef struct vs_ctx vs_ctx;

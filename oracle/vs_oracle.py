@@ -132,6 +132,29 @@ def estimate(q_rows: np.ndarray, k: np.ndarray, e: int, base: float, scale: floa
     return lse, vert, slash, a
 
 
+def estimate_probs_dca(q_rows: np.ndarray, k: np.ndarray, e: int, base: float, scale: float,
+                       dca: tuple):
+    """The estimation rows' attention at DCA positions (dca = (C, W)): the softmax
+    the prefill applies to these rows over all keys j <= i ([QW] Length
+    Extrapolation: each (query, key) pair scored at the positions of its class).
+    Used by the recall-at-DCA-positions variant of refinement; selection itself
+    keeps the continuous positions of `estimate`. Returns (lse (nr,), A (nr, e))."""
+    C, W = dca
+    nr = q_rows.shape[0]
+    rows = np.arange(e - nr, e)
+    kr = rope(k[:e], np.arange(e) % (C - W), base)
+    s = np.full((nr, e), _NEG_INF)
+    for r, i in enumerate(rows):
+        j = np.arange(i + 1)
+        pq, _ = dca_positions(int(i), j, C, W)
+        qv = {int(p): rope(q_rows[r : r + 1], np.array([p]), base)[0] for p in np.unique(pq)}
+        qj = np.stack([qv[int(p)] for p in pq])
+        s[r, : i + 1] = scale * np.einsum("jd,jd->j", qj, kr[: i + 1])
+    mx = s.max(axis=1, keepdims=True)
+    lse = (mx + np.log(np.exp(s - mx).sum(axis=1, keepdims=True)))[:, 0]
+    return lse, np.exp(s - lse[:, None])
+
+
 # ----------------------------------------------------------------------------- selection  [QW Sparse Attention]
 def topk_sorted(score: np.ndarray, k: int) -> np.ndarray:
     """Indices of the k largest scores, ranked by (score descending, index

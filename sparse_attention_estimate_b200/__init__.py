@@ -44,7 +44,8 @@ class AttnCfg(ctypes.Structure):
     _fields_ = [("hq", ctypes.c_int32), ("hkv", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("last_q", ctypes.c_int32), ("softmax_scale", ctypes.c_float),
                 ("rope_base", ctypes.c_double), ("dca_enabled", ctypes.c_int32),
-                ("dca_chunk_size", ctypes.c_int64), ("dca_local_window", ctypes.c_int64)]
+                ("dca_chunk_size", ctypes.c_int64), ("dca_local_window", ctypes.c_int64),
+                ("refine_dca_positions", ctypes.c_int32)]
 
 
 _lib = None
@@ -124,6 +125,7 @@ class Config:
     last_q: int = 64
     dca_chunk: Optional[int] = None
     dca_window: Optional[int] = None
+    refine_dca_positions: bool = False  # recall at DCA positions (DCA only)
 
     def to_c(self) -> AttnCfg:
         c = AttnCfg()
@@ -134,6 +136,7 @@ class Config:
         c.dca_chunk_size = self.dca_chunk or 0
         c.dca_local_window = (self.dca_window if self.dca_window is not None else
                               (self.dca_chunk // 32 if self.dca_chunk else 0))
+        c.refine_dca_positions = 1 if self.refine_dca_positions else 0
         return c
 
 

@@ -64,6 +64,7 @@ Layout make_layout(const vs_attn_cfg& cfg, int64_t max_seq, int64_t max_chunk) {
   L.q_rot = take(static_cast<size_t>(L.nvar) * hq * L.rows_pad * kD * 2);
   L.q_est = take(static_cast<size_t>(hkv) * L.ntile * kTile * kD * 2);
   L.est_ml = take(static_cast<size_t>(L.nsplit_max) * hq * kEstRows * 2 * sizeof(float));
+  L.lse_dca = take(static_cast<size_t>(hq) * kEstRows * sizeof(float));
   L.part_v = take(static_cast<size_t>(hq) * 2 * L.e_pad * sizeof(float));
   L.part_s = take(static_cast<size_t>(hq) * 4 * (L.e_pad + 256) * sizeof(float));
   L.thr = take(static_cast<size_t>(hq) * 2 * kMaxLevels * 2 * sizeof(uint32_t));
@@ -117,11 +118,6 @@ using namespace vs;
 // ------------------------------------------------------------------ validation helpers
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-#define VS_REQUIRE(cond, code, ...)          \
-  do {                                       \
-    if (!(cond)) return set_error(code, __VA_ARGS__); \
-  } while (0)
-
 static vs_status check_cfg(const vs_attn_cfg* cfg) {
   VS_REQUIRE(cfg, VS_ERR_INVALID_ARG, "cfg is NULL");
   VS_REQUIRE(cfg->head_dim == kD, VS_ERR_UNSUPPORTED, "head_dim %d: only 128 is supported",
@@ -163,11 +159,6 @@ static vs_status check_tensor(const void* p, const char* name) {
   return VS_OK;
 }
 
-#define VS_TRY(expr)                 \
-  do {                               \
-    vs_status _s = (expr);           \
-    if (_s != VS_OK) return _s;      \
-  } while (0)
 
 // ------------------------------------------------------------------ context
 extern "C" vs_status vs_workspace_size(const vs_attn_cfg* cfg, int64_t max_seq, int64_t max_chunk,
@@ -367,7 +358,10 @@ extern "C" vs_status vs_refine(vs_ctx* c, const uint16_t* q, int64_t q_rows, int
   VS_TRY(prepare_estimation(c, q, q_rows, q_pos0, k, k_rows, e, st, &nr));
   VS_TRY(run_thresholds(c, vert, slash, e_ld, e, kv_budget, ks_budget, nlev, st));
   VS_TRY(run_levels(c, vert, slash, e_ld, e, nlev, st));
-  VS_TRY(run_recall_hist(c, e, nr, lse, nlev, st));
+  if (c->cfg.refine_dca_positions && c->dca.enabled)
+    VS_TRY(run_recall_hist_dca(c, q, q_rows, q_pos0, k, k_rows, e, nr, nlev, st));
+  else
+    VS_TRY(run_recall_hist(c, e, nr, lse, nlev, st));
   VS_TRY(run_refine_decide(c, e, nr, nlev, tau, kv_budget, ks_budget, recall, st));
   return run_compact(c, e, ws_ptr<int32_t>(c, c->L.choice), v_idx, cap_v, v_cnt, s_off, cap_s,
                      s_cnt, st);

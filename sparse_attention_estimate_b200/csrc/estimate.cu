@@ -42,7 +42,9 @@ struct EstParams {
   int64_t e_pad;      // row stride of the partial arrays
   int nr;             // estimation rows per head
   int g, ntile, hq;
-  int nblk;           // key blocks in [0, e)
+  int nblk;           // end of this launch's key-block range (blocks [blk0, nblk))
+  int blk0;           // first key block of this launch
+  int split0;         // index of this launch's first split in the partial outputs
   int bps;            // key blocks per split
   float scale_log2;   // softmax_scale * log2(e)
   float* part_ml;     // kLse: [nsplit][hq*64][2] (max, sum) in log2 units
@@ -115,8 +117,8 @@ __global__ void __launch_bounds__(kEstThreads, 1)
   EstSmem& s = *reinterpret_cast<EstSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int G = blockIdx.y, split = blockIdx.x;
-  const int b_begin = split * p.bps;
+  const int G = blockIdx.y, split = p.split0 + static_cast<int>(blockIdx.x);
+  const int b_begin = p.blk0 + static_cast<int>(blockIdx.x) * p.bps;
   const int b_end = min(b_begin + p.bps, p.nblk);
   const int nb = b_end - b_begin;
   volatile int* abort_word = &s.abort_word;
@@ -415,21 +417,29 @@ __global__ void sums_fixup_kernel(const float* __restrict__ part_v, const float*
   slash[static_cast<int64_t>(h) * e_ld + d] = acc;
 }
 
-static vs_status launch_est(vs_ctx* c, int mode, int64_t e, int nr, const float* lse, int nlev,
-                            int* nsplit_out, cudaStream_t st) {
+// One estimation-kernel launch over key blocks [blk0, blk1) with the rotated rows
+// in q_buf and the rotated keys in k_buf; its splits write partial outputs from
+// index split0 on. *nsplit_out gets the number of splits used.
+static vs_status launch_est_range(vs_ctx* c, int mode, int64_t e, int nr, const float* lse, int nlev,
+                                  int blk0, int blk1, int split0, int max_splits, size_t q_buf,
+                                  size_t k_buf, int* nsplit_out, cudaStream_t st) {
   const int hkv = c->cfg.hkv, g = c->cfg.hq / c->cfg.hkv;
-  const int nblk = static_cast<int>(ceil_div(e, kTile));
+  const int nblk = blk1 - blk0;
+  if (nblk <= 0) {
+    *nsplit_out = 0;
+    return VS_OK;
+  }
   int nsplit = std::max(1, c->num_sms / hkv);
   nsplit = std::min(nsplit, nblk);
-  nsplit = std::min(nsplit, c->L.nsplit_max);
+  nsplit = std::min(nsplit, max_splits);
   const int bps = static_cast<int>(ceil_div(nblk, nsplit));
   nsplit = static_cast<int>(ceil_div(nblk, bps));
   *nsplit_out = nsplit;
   CUtensorMap tmQ, tmK;
-  vs_status s = make_tmap_rows(&tmQ, c->ws + c->L.q_est, hkv, static_cast<int64_t>(c->L.ntile) * kTile,
+  vs_status s = make_tmap_rows(&tmQ, c->ws + q_buf, hkv, static_cast<int64_t>(c->L.ntile) * kTile,
                                static_cast<int64_t>(c->L.ntile) * kTile, kTile);
   if (s != VS_OK) return s;
-  s = make_tmap_rows(&tmK, c->ws + c->L.k_cont, hkv, e, c->max_seq, kTile);
+  s = make_tmap_rows(&tmK, c->ws + k_buf, hkv, e, c->max_seq, kTile);
   if (s != VS_OK) return s;
   EstParams p{};
   p.e = e;
@@ -439,7 +449,9 @@ static vs_status launch_est(vs_ctx* c, int mode, int64_t e, int nr, const float*
   p.g = g;
   p.ntile = c->L.ntile;
   p.hq = c->cfg.hq;
-  p.nblk = nblk;
+  p.nblk = blk1;
+  p.blk0 = blk0;
+  p.split0 = split0;
   p.bps = bps;
   p.scale_log2 = c->cfg.softmax_scale * kLog2e;
   p.part_ml = ws_ptr<float>(c, c->L.est_ml);
@@ -452,7 +464,6 @@ static vs_status launch_est(vs_ctx* c, int mode, int64_t e, int nr, const float*
   p.dc = dev_common(c);
   const size_t smem = sizeof(EstSmem) + 1024;
   dim3 grid(nsplit, hkv);
-  cudaError_t err;
   if (mode == kLse) {
     cudaFuncSetAttribute(est_kernel<kLse>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     est_kernel<kLse><<<grid, kEstThreads, smem, st>>>(tmQ, tmK, p);
@@ -463,8 +474,15 @@ static vs_status launch_est(vs_ctx* c, int mode, int64_t e, int nr, const float*
     cudaFuncSetAttribute(est_kernel<kRecall>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     est_kernel<kRecall><<<grid, kEstThreads, smem, st>>>(tmQ, tmK, p);
   }
-  (void)err;
   return launched("est_kernel launch");
+}
+
+// All key blocks of [0, e) with continuous positions (estimation rows in q_est,
+// keys in the continuous rotated cache).
+static vs_status launch_est(vs_ctx* c, int mode, int64_t e, int nr, const float* lse, int nlev,
+                            int* nsplit_out, cudaStream_t st) {
+  return launch_est_range(c, mode, e, nr, lse, nlev, 0, static_cast<int>(ceil_div(e, kTile)), 0,
+                          c->L.nsplit_max, c->L.q_est, c->L.k_cont, nsplit_out, st);
 }
 
 vs_status run_estimate(vs_ctx* c, const uint16_t* q, int64_t q_rows, int64_t q_pos0,
@@ -490,6 +508,62 @@ vs_status run_estimate(vs_ctx* c, const uint16_t* q, int64_t q_rows, int64_t q_p
       ws_ptr<float>(c, c->L.part_v), ws_ptr<float>(c, c->L.part_s), e, e - nr, c->L.e_pad, cover,
       vert, slash, e_ld);
   return launched("sums_fixup_kernel launch");
+}
+
+// The recall histogram from the estimation rows' attention at DCA positions (the
+// attention the prefill computes) instead of continuous ones. The rows R lie in one
+// DCA chunk b, so each 128-key block has one class for all of them (S % 128 == 0):
+// keys in chunk b are intra, in chunk b-1 successive, before that inter. Per class,
+// the rows are rotated at that class's query positions and the kernel runs over the
+// class's key blocks against the DCA-rotated keys: first the lse pass (combined over
+// all classes' splits), then the histogram pass with that lse.
+vs_status run_recall_hist_dca(vs_ctx* c, const uint16_t* q, int64_t q_rows, int64_t q_pos0,
+                              const uint16_t* k, int64_t k_rows, int64_t e, int nr, int nlev,
+                              cudaStream_t st) {
+  const int64_t S = c->dca.S;
+  VS_REQUIRE(S % kTile == 0, VS_ERR_UNSUPPORTED,
+             "recall at DCA positions needs the DCA stride C - W to be a multiple of 128");
+  const int64_t b = (e - 1) / S;
+  VS_REQUIRE((e - nr) / S == b, VS_ERR_UNSUPPORTED,
+             "the estimation rows straddle a DCA chunk boundary");
+  VS_TRY(ensure_keys_rotated(c, k, k_rows, e, true, st));
+  const int nblk = static_cast<int>(ceil_div(e, kTile));
+  int lo[3], hi[3];  // key-block ranges by class: 0 intra, 1 successive, 2 inter
+  lo[2] = 0;
+  hi[2] = b >= 2 ? static_cast<int>((b - 1) * S / kTile) : 0;
+  lo[1] = hi[2];
+  hi[1] = b >= 1 ? static_cast<int>(b * S / kTile) : 0;
+  lo[0] = hi[1];
+  hi[0] = nblk;
+  const int g = c->cfg.hq / c->cfg.hkv;
+  auto rotate = [&](int cls) {
+    return launch_rope_rows(c, reinterpret_cast<const bf16*>(q), q_rows, e - nr - q_pos0,
+                            ws_ptr<bf16>(c, c->L.q_est), 0, 0, g,
+                            static_cast<int64_t>(c->L.ntile) * kTile, kEstRows, nr, c->cfg.hq,
+                            e - nr, 2 + cls, st);
+  };
+  float* lse_dca = ws_ptr<float>(c, c->L.lse_dca);
+  int total[2] = {0, 0};
+  for (int pass = 0; pass < 2; ++pass) {
+    for (int cls = 2; cls >= 0; --cls) {
+      if (hi[cls] <= lo[cls]) continue;
+      VS_TRY(rotate(cls));
+      const int budget = std::max(1, (c->L.nsplit_max - total[pass]) / (cls + 1));
+      int ns = 0;
+      VS_TRY(launch_est_range(c, pass == 0 ? kLse : kRecall, e, nr, pass == 0 ? nullptr : lse_dca,
+                              pass == 0 ? 0 : nlev, lo[cls], hi[cls], total[pass], budget,
+                              c->L.q_est, c->L.k_dca, &ns, st));
+      total[pass] += ns;
+    }
+    if (pass == 0) {
+      const int n = c->cfg.hq * kEstRows;
+      lse_combine_kernel<<<ceil_div(n, 256), 256, 0, st>>>(ws_ptr<float>(c, c->L.est_ml), total[0],
+                                                          c->cfg.hq, nr, lse_dca);
+      VS_TRY(launched("lse_combine_kernel launch"));
+    }
+  }
+  c->hist_nsplit = total[1];
+  return VS_OK;
 }
 
 vs_status run_recall_hist(vs_ctx* c, int64_t e, int nr, const float* lse, int nlev,

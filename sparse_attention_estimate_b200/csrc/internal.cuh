@@ -53,6 +53,7 @@ struct Layout {
   size_t q_rot;               // rotated chunk queries [nvar][hq][rows_pad][128]
   size_t q_est;               // rotated estimation rows [hkv][ntile*128][128]
   size_t est_ml;              // lse partials [nsplit_max][hq*64][2]
+  size_t lse_dca;             // estimation rows' lse at DCA positions [hq][64]
   size_t part_v;              // vertical partial sums [hq][2][e_pad]
   size_t part_s;              // slash partial sums [hq][2 halves][2 lo/hi][e_pad + 128]
   size_t thr;                 // selection thresholds [hq][2][kMaxLevels] (key, take)
@@ -107,6 +108,18 @@ inline DevCommon dev_common(vs_ctx* c) { return DevCommon{c->err, c->wait_ns}; }
 
 // Error reporting (thread-local message).
 vs_status set_error(vs_status s, const char* fmt, ...);
+
+// Host-side checks: return the status (with the thread's error message set) from
+// the enclosing function.
+#define VS_REQUIRE(cond, code, ...)                   \
+  do {                                                \
+    if (!(cond)) return set_error(code, __VA_ARGS__); \
+  } while (0)
+#define VS_TRY(expr)            \
+  do {                          \
+    vs_status _s = (expr);      \
+    if (_s != VS_OK) return _s; \
+  } while (0)
 vs_status cuda_check(cudaError_t e, const char* what);
 
 // TMA descriptor for a [heads][rows][128] bf16 tensor: box of 64 columns x box_rows rows x 1 head,
@@ -128,6 +141,9 @@ vs_status launch_dca_remap(vs_ctx* c, int64_t pos0, int64_t n, int32_t* pk, int3
 vs_status run_estimate(vs_ctx* c, const uint16_t* q, int64_t q_rows, int64_t q_pos0,
                        const uint16_t* k, int64_t k_rows, int64_t e, float* vert, float* slash,
                        int64_t e_ld, float* lse, cudaStream_t st);
+vs_status run_recall_hist_dca(vs_ctx* c, const uint16_t* q, int64_t q_rows, int64_t q_pos0,
+                              const uint16_t* k, int64_t k_rows, int64_t e, int nr, int nlev,
+                              cudaStream_t st);
 vs_status run_recall_hist(vs_ctx* c, int64_t e, int nr, const float* lse, int nlev,
                           cudaStream_t st);
 // select.cu

@@ -180,6 +180,41 @@ def test_refine_matches_oracle(case, tau):
         assert ctx.status() == vsb.VS_OK
 
 
+@pytest.mark.parametrize("tau", [0.3, 0.9, 0.999])
+def test_refine_recall_at_dca_positions(case, tau):
+    """Refinement whose recall comes from the estimation rows' attention at DCA
+    positions (selection still on continuous positions), against the oracle's
+    refinement driven by estimate_probs_dca."""
+    name, w, dca, dev, cpu, _ = case
+    if dca is None:
+        pytest.skip("no DCA")
+    ctx = make_ctx(w, dca=dca, refine_dca_positions=True)
+    scale = scale_of(w)
+    for cs, e in _chunks(w):
+        qc = dev["q"][:, cs:e].contiguous()
+        vert, slash, lse = ctx.estimate(qc, cs, dev["k"], e)
+        kvb = torch.full((w.hq,), w.kv_budget, dtype=torch.int32, device="cuda")
+        ksb = torch.full((w.hq,), w.ks_budget, dtype=torch.int32, device="cuda")
+        sets, recall = ctx.refine(qc, cs, dev["k"], e, vert, slash, lse, tau, kvb, ksb)
+        assert ctx.status() == vsb.VS_OK
+        V, S = sets_to_lists(sets)
+        kvb, ksb, recall = kvb.cpu().numpy(), ksb.cpu().numpy(), recall.cpu().numpy()
+        gv, gs = f64(vert), f64(slash)
+        nr = min(w.last_q, e - cs)
+        rows = np.arange(e - nr, e)
+        for h in range(w.hq):
+            ov, osl = vo.select(gv[h], gs[h], int(kvb[h]), int(ksb[h]))
+            assert np.array_equal(V[h], ov) and np.array_equal(S[h], osl), (name, cs, h)
+            qh, kh = cpu["q"][h, e - nr : e], cpu["k"][h // w.group]
+            _, ovv, oss, _ = vo.estimate(qh, kh, e, w.rope_base, scale)
+            _, a_dca = vo.estimate_probs_dca(qh, kh, e, w.rope_base, scale, dca)
+            okv, oks, _, _, orc, trace = vo.refine(a_dca, rows, ovv, oss, w.kv_budget, w.ks_budget, tau)
+            if (okv, oks) != (int(kvb[h]), int(ksb[h])):
+                assert any(abs(rc - tau) < TAU_SLACK for _, _, rc in trace), (name, cs, h, trace, kvb[h])
+            else:
+                assert abs(recall[h] - orc) < 1e-4, (name, cs, h, recall[h], orc)
+
+
 def _random_sets(rng, hq, e, pv, ps, force0=True):
     V, S = [], []
     for _ in range(hq):

@@ -420,6 +420,29 @@ def test_calibration_budgets(rng):
             assert r["kv"] == min(kv[h], c["e"]) and r["ks"] == min(ks[h], c["e"])
 
 
+def test_estimation_at_dca_positions(rng):
+    """Recall-at-DCA-positions variant: the estimation rows' DCA attention has the
+    lse of the dense full-mask DCA attention of the same rows (an independent code
+    path), rows sum to one, and with C >= N every pair keeps its continuous
+    positions, so it equals the continuous estimation exactly."""
+    n, d, nr = 90, 16, 6
+    q = _bf16_array(rng, (nr, d), 2.0)
+    k = _bf16_array(rng, (n, d), 2.0)
+    v = _bf16_array(rng, (n, d))
+    scale = 1 / math.sqrt(d)
+    rows = np.arange(n - nr, n)
+    dca = (40, 8)
+    lse, a = vo.estimate_probs_dca(q, k, n, BASE, scale, dca)
+    assert np.allclose(a.sum(axis=1), 1.0, rtol=0, atol=1e-12)
+    full = np.ones(n, dtype=bool)
+    _, lse_att = vo.attention_rows_dense(q, rows, k, v, n, full, full, BASE, scale, dca)
+    assert np.allclose(lse, lse_att, rtol=0, atol=1e-12)
+    lse_c, _, _, a_c = vo.estimate(q, k, n, BASE, scale)
+    lse_w, a_w = vo.estimate_probs_dca(q, k, n, BASE, scale, (128, 16))
+    assert np.array_equal(a_w, a_c) and np.array_equal(lse_w, lse_c)
+    assert not np.allclose(a, a_c, rtol=0, atol=1e-6)  # DCA positions do change the scores
+
+
 # ------------------------------------------------------------------ sensitivity
 MUTANTS = {
     "rope_sign": lambda x1, x2, c, s: (x1 * c + x2 * s, x2 * c - x1 * s),
