@@ -513,18 +513,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int c = 0; c < 128; ++c)
           if (!((mw[c >> 5] >> (c & 31)) & 1u)) sv[c] = -INFINITY;
       }
-      float mx[16];
+      // row max of the raw scores: 8 chains of 3-input max (scale > 0 keeps the order)
+      float mx[8];
 #pragma unroll
-      for (int x = 0; x < 16; ++x) mx[x] = fmaxf(sv[x], sv[x + 16]);
+      for (int x = 0; x < 8; ++x) {
+        mx[x] = fmax3(sv[x], sv[x + 8], sv[x + 16]);
 #pragma unroll
-      for (int c = 32; c < 128; c += 16)
-#pragma unroll
-        for (int x = 0; x < 16; ++x) mx[x] = fmaxf(mx[x], sv[c + x]);
-#pragma unroll
-      for (int w2 = 8; w2 >= 1; w2 >>= 1)
-#pragma unroll
-        for (int x = 0; x < w2; ++x) mx[x] = fmaxf(mx[x], mx[x + w2]);
-      const float mblk = mx[0] * p.scale_log2;
+        for (int c = 24; c < 120; c += 16) mx[x] = fmax3(mx[x], sv[x + c], sv[x + c + 8]);
+        mx[x] = fmaxf(mx[x], sv[x + 120]);
+      }
+      const float mblk =
+          fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * p.scale_log2;
       useful += __popc(mw[0]) + __popc(mw[1]) + __popc(mw[2]) + __popc(mw[3]);
       // lazy rescale: move the reference max only when it grows by > 2^8
       const float m_new = fmaxf(m_run, mblk);
@@ -546,24 +545,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         l_run *= f;
         m_run = m_new;
       }
+      // p = exp2(s * scale * log2(e) - m): the arguments of two columns per packed
+      // fp32x2 FMA, one MUFU exp2 per element, the row sum over 4 packed chains, P as
+      // bf16 pairs (issue slots, not a pipe, bound this warp's loop)
       const float nm = (m_run == -INFINITY) ? 0.f : -m_run;
-      float ls[8];
-#pragma unroll
-      for (int x = 0; x < 8; ++x) ls[x] = 0.f;
+      const uint64_t sc2 = f32x2_pack(p.scale_log2, p.scale_log2), nm2 = f32x2_pack(nm, nm);
+      uint64_t ls2[4] = {0ull, 0ull, 0ull, 0ull};
       uint32_t pk[64];
 #pragma unroll
       for (int c = 0; c < 64; ++c) {
-        const float p0 = ex2a(fmaf(sv[2 * c], p.scale_log2, nm));
-        const float p1 = ex2a(fmaf(sv[2 * c + 1], p.scale_log2, nm));
-        ls[(2 * c) & 7] += p0;
-        ls[(2 * c + 1) & 7] += p1;
+        float a0, a1;
+        f32x2_unpack(f32x2_fma(f32x2_pack(sv[2 * c], sv[2 * c + 1]), sc2, nm2), a0, a1);
+        const float p0 = ex2a(a0), p1 = ex2a(a1);
+        ls2[c & 3] = f32x2_add(ls2[c & 3], f32x2_pack(p0, p1));
         pk[c] = pack_bf16x2(p0, p1);
       }
+      float lsum = 0.f;
 #pragma unroll
-      for (int w2 = 4; w2 >= 1; w2 >>= 1)
-#pragma unroll
-        for (int x = 0; x < w2; ++x) ls[x] += ls[x + w2];
-      l_run += ls[0];
+      for (int x = 0; x < 4; ++x) {
+        float u0, u1;
+        f32x2_unpack(ls2[x], u0, u1);
+        lsum += u0 + u1;
+      }
+      l_run += lsum;
       tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(pk));
       tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
       tmem_wait_st();
