@@ -21,9 +21,10 @@
 //             O_t += P_t V (TS: P read from tensor memory, V MN-major in smem).
 //  warps 4-7  softmax of tile 0, warps 8-11 of tile 1; one thread per query row:
 //             tcgen05.ld of S, element mask from the vertical / slash bitmaps,
-//             online softmax in fp32 with exp2 and a lazy rescale of O (only when
-//             the running max grows by more than 2^8), P as bf16 written back
-//             into S's tensor-memory columns.
+//             online softmax in fp32 with exp2, optimistic (a row with a reference
+//             max skips the max pass unless the block's sum exceeds 2^16) and a lazy
+//             rescale of O (only when the running max grows by more than 2^8), P as
+//             bf16 written back into S's tensor-memory columns.
 // Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256,384),
 // O1 [384,512); P_t aliases the first 64 columns of S_t. The next S_t MMA is
 // issued after the PV MMA that reads P_t; tcgen05 MMAs of one thread execute in
@@ -43,6 +44,10 @@ constexpr uint32_t kRegsControl = 112, kRegsSoftmax = 192;
 static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= 384 * 168, "register split exceeds the launch");
 constexpr float kLog2eA = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// A block exponentiated against the row's reference max without a max pass is kept
+// when its row sum stays at or below this (every p <= 2^16, far inside bf16 and the
+// fp32 accumulators); otherwise it is redone with its own max.
+constexpr float kOptimisticSum = 65536.0f;
 constexpr int kDevErrIndex = 4;            // an index list held an out-of-range entry
 
 // ---------------------------------------------------------------- bitmaps
@@ -498,74 +503,95 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&s.s_full[t], j & 1, abort_word, p.dc.err));
       if (!ok) break;
       tc_fence_after_sync();
-      float sv[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t raw[32];
-        tmem_ld32(tS + c * 32, raw);
-#pragma unroll
-        for (int x = 0; x < 32; ++x) sv[c * 32 + x] = __uint_as_float(raw[x]);
-      }
-      tmem_wait_ld();
-      const bool all_on = __all_sync(0xffffffffu, (mw[0] & mw[1] & mw[2] & mw[3]) == 0xFFFFFFFFu);
-      if (!all_on) {
-#pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (!((mw[c >> 5] >> (c & 31)) & 1u)) sv[c] = -INFINITY;
-      }
-      // row max of the raw scores: 8 chains of 3-input max (scale > 0 keeps the order)
-      float mx[8];
-#pragma unroll
-      for (int x = 0; x < 8; ++x) {
-        mx[x] = fmax3(sv[x], sv[x + 8], sv[x + 16]);
-#pragma unroll
-        for (int c = 24; c < 120; c += 16) mx[x] = fmax3(mx[x], sv[x + c], sv[x + c + 8]);
-        mx[x] = fmaxf(mx[x], sv[x + 120]);
-      }
-      const float mblk =
-          fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * p.scale_log2;
       useful += __popc(mw[0]) + __popc(mw[1]) + __popc(mw[2]) + __popc(mw[3]);
-      // lazy rescale: move the reference max only when it grows by > 2^8
-      const float m_new = fmaxf(m_run, mblk);
-      const bool need = m_new > m_run + kRescaleThreshold;
-      const float f = need ? ex2a(m_run - m_new) : 1.0f;  // 0 when m_run = -inf
-      if (j > 0 && __any_sync(0xffffffffu, need && m_run != -INFINITY)) {
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + c * 32, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * f);
-          tmem_st32(tO + c * 32, o);
-        }
-        tmem_wait_st();
-      }
-      if (need) {
-        l_run *= f;
-        m_run = m_new;
-      }
-      // p = exp2(s * scale * log2(e) - m): the arguments of two columns per packed
-      // fp32x2 FMA, one MUFU exp2 per element, the row sum over 4 packed chains, P as
-      // bf16 pairs (issue slots, not a pipe, bound this warp's loop)
-      const float nm = (m_run == -INFINITY) ? 0.f : -m_run;
-      const uint64_t sc2 = f32x2_pack(p.scale_log2, p.scale_log2), nm2 = f32x2_pack(nm, nm);
-      uint64_t ls2[4] = {0ull, 0ull, 0ull, 0ull};
+      // Optimistic softmax: a row that already has a reference max is exponentiated
+      // against it without a max pass. A block whose row sum exceeds 2^16 (so some p
+      // may exceed 2^16) is redone from S, which stays in tensor memory until P is
+      // stored, with its true max and the lazy-rescale rule; so is every block of a
+      // warp with a row still without reference.
+      bool optimistic = __all_sync(0xffffffffu, m_run != -INFINITY);
       uint32_t pk[64];
-#pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        float a0, a1;
-        f32x2_unpack(f32x2_fma(f32x2_pack(sv[2 * c], sv[2 * c + 1]), sc2, nm2), a0, a1);
-        const float p0 = ex2a(a0), p1 = ex2a(a1);
-        ls2[c & 3] = f32x2_add(ls2[c & 3], f32x2_pack(p0, p1));
-        pk[c] = pack_bf16x2(p0, p1);
-      }
       float lsum = 0.f;
+#pragma unroll 1
+      for (int attempt = 0; attempt < 2; ++attempt) {
+        // the row's 128 scores: four tcgen05.ld and one wait
+        float sv[128];
 #pragma unroll
-      for (int x = 0; x < 4; ++x) {
-        float u0, u1;
-        f32x2_unpack(ls2[x], u0, u1);
-        lsum += u0 + u1;
+        for (int c = 0; c < 4; ++c) {
+          uint32_t raw[32];
+          tmem_ld32(tS + c * 32, raw);
+#pragma unroll
+          for (int x = 0; x < 32; ++x) sv[c * 32 + x] = __uint_as_float(raw[x]);
+        }
+        tmem_wait_ld();
+        // element mask; blocks where every lane keeps all 128 keys skip the selects
+        const bool all_on = __all_sync(0xffffffffu, (mw[0] & mw[1] & mw[2] & mw[3]) == 0xFFFFFFFFu);
+        if (!all_on) {
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (!((mw[c >> 5] >> (c & 31)) & 1u)) sv[c] = -INFINITY;
+        }
+        if (!optimistic) {
+          // row max of the raw scores: 8 chains of 3-input max (scale > 0 keeps the order)
+          float mx[8];
+#pragma unroll
+          for (int x = 0; x < 8; ++x) {
+            mx[x] = fmax3(sv[x], sv[x + 8], sv[x + 16]);
+#pragma unroll
+            for (int c = 24; c < 120; c += 16) mx[x] = fmax3(mx[x], sv[x + c], sv[x + c + 8]);
+            mx[x] = fmaxf(mx[x], sv[x + 120]);
+          }
+          const float mblk =
+              fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) *
+              p.scale_log2;
+          // lazy rescale: move the reference max only when it grows by > 2^8
+          const float m_new = fmaxf(m_run, mblk);
+          const bool need = m_new > m_run + kRescaleThreshold;
+          const float f = need ? ex2a(m_run - m_new) : 1.0f;  // 0 when m_run = -inf
+          // O_t holds PV_t(j-1) complete: S_t(j) was committed after it
+          if (j > 0 && __any_sync(0xffffffffu, need && m_run != -INFINITY)) {
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+              uint32_t o[32];
+              tmem_ld32(tO + c * 32, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * f);
+              tmem_st32(tO + c * 32, o);
+            }
+            tmem_wait_st();
+          }
+          if (need) {
+            l_run *= f;
+            m_run = m_new;
+          }
+        }
+        // p = exp2(s * scale * log2(e) - m): the arguments of two columns per packed
+        // fp32x2 FMA, one MUFU exp2 per element, the row sum over 4 packed chains, P as
+        // bf16 pairs (issue slots, not a pipe, bound this warp's loop)
+        const float nm = (m_run == -INFINITY) ? 0.f : -m_run;
+        const uint64_t sc2 = f32x2_pack(p.scale_log2, p.scale_log2), nm2 = f32x2_pack(nm, nm);
+        uint64_t ls2[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          float a0, a1;
+          f32x2_unpack(f32x2_fma(f32x2_pack(sv[2 * c], sv[2 * c + 1]), sc2, nm2), a0, a1);
+          const float p0 = ex2a(a0), p1 = ex2a(a1);
+          ls2[c & 3] = f32x2_add(ls2[c & 3], f32x2_pack(p0, p1));
+          pk[c] = pack_bf16x2(p0, p1);
+        }
+        lsum = 0.f;
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+          float u0, u1;
+          f32x2_unpack(ls2[x], u0, u1);
+          lsum += u0 + u1;
+        }
+        if (optimistic && __any_sync(0xffffffffu, lsum > kOptimisticSum)) {
+          optimistic = false;
+          continue;
+        }
+        break;
       }
       l_run += lsum;
       tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(pk));
