@@ -395,23 +395,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const int st1 = (j + 1) & 1;
             const int64_t kb1 = more ? static_cast<int64_t>(ent1 & 0xFFFFFF) * kTile : 0;
             ent1 = j + 2 < n ? ld_keep_s32(list + j + 2) : 0;
+            const int c0 = more ? dca_class(R0, kb1, p.dca) : cls[0];
+            const int c1 = more ? dca_class(R0 + kTile, kb1, p.dca) : cls[1];
+            // V(j) and K(j+1) normally landed long ago: wait for them before P_0(j), so
+            // that PV_t(j) and S_t(j + 1) go to the tensor pipe back to back once P_t(j)
+            // is stored (the pipe runs dry while this thread does anything else)
+            ok = mbar_wait(&s.v_full[st], (j >> 1) & 1, abort_word, p.dc.err) &&
+                 (!more || mbar_wait(&s.k_full[st1], ((j + 1) >> 1) & 1, abort_word, p.dc.err));
             // tile 0
-            ok = mbar_wait(&s.p_full[0], j & 1, abort_word, p.dc.err) &&
-                 mbar_wait(&s.v_full[st], (j >> 1) & 1, abort_word, p.dc.err);
+            ok = ok && mbar_wait(&s.p_full[0], j & 1, abort_word, p.dc.err);
             if (!ok) break;
             tc_fence_after_sync();
             issue_pv(0, st, j > 0);
             if (more) {
-              const int c = dca_class(R0, kb1, p.dca);
-              if (c != cls[0]) {
+              if (c0 != cls[0]) {  // the tile's DCA class changes: wait for Q_0 at the new rotation
                 mma_commit(&s.q_empty[0]);
                 ok = mbar_wait(&s.q_full[0], qph[0] & 1, abort_word, p.dc.err);
                 ++qph[0];
-                cls[0] = c;
+                cls[0] = c0;
+                if (!ok) break;
+                tc_fence_after_sync();
               }
-              ok = ok && mbar_wait(&s.k_full[st1], ((j + 1) >> 1) & 1, abort_word, p.dc.err);
-              if (!ok) break;
-              tc_fence_after_sync();
               issue_qk(0, st1);
               mma_commit(&s.s_full[0]);
             }
@@ -422,15 +426,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             issue_pv(1, st, j > 0);
             mma_commit(&s.v_empty[st]);
             if (more) {
-              const int c = dca_class(R0 + kTile, kb1, p.dca);
-              if (c != cls[1]) {
+              if (c1 != cls[1]) {
                 mma_commit(&s.q_empty[1]);
                 ok = mbar_wait(&s.q_full[1], qph[1] & 1, abort_word, p.dc.err);
                 ++qph[1];
-                cls[1] = c;
+                cls[1] = c1;
+                if (!ok) break;
+                tc_fence_after_sync();
               }
-              if (!ok) break;
-              tc_fence_after_sync();
               issue_qk(1, st1);
               mma_commit(&s.s_full[1]);
               mma_commit(&s.k_empty[st1]);
