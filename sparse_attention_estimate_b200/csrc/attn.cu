@@ -361,22 +361,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           cls[0] = dca_class(R0, kb0, p.dca);
           cls[1] = dca_class(R0 + kTile, kb0, p.dca);
           int32_t ent1 = n > 1 ? list[1] : 0;  // entry of block j + 1, read a block ahead
+          // descriptor words of the operand tiles (K-major Q and K, MN-major V; 128-byte swizzle)
+          const uint32_t dhi = smem_desc_sw128_hi(1024);
+          const uint32_t qlo[2] = {smem_desc_sw128_lo(smem_u32(&s.q[0][0][0]), 16),
+                                   smem_desc_sw128_lo(smem_u32(&s.q[1][0][0]), 16)};
+          const uint32_t klo[2] = {smem_desc_sw128_lo(smem_u32(&s.k[0][0][0]), 16),
+                                   smem_desc_sw128_lo(smem_u32(&s.k[1][0][0]), 16)};
+          const uint32_t vlo[2] = {smem_desc_sw128_lo(smem_u32(&s.v[0][0][0]), kTileBytes),
+                                   smem_desc_sw128_lo(smem_u32(&s.v[1][0][0]), kTileBytes)};
           auto issue_qk = [&](int t, int st) {
-            const uint32_t qa = smem_u32(&s.q[t][0][0]);
-            const uint32_t ka = smem_u32(&s.k[st][0][0]);
+            const uint32_t a = qlo[t], b = klo[st];
   #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
-              const uint32_t off = (kk >> 2) * kTileBytes + (kk & 3) * 32;
-              mma_bf16_ss(tS[t], smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024),
-                          id_qk, kk > 0 ? 1u : 0u);
+              const uint32_t off = ((kk >> 2) * kTileBytes + (kk & 3) * 32) >> 4;  // K-step of 16 columns
+              mma_bf16_ss_w(tS[t], a + off, b + off, dhi, id_qk, kk > 0 ? 1u : 0u);
             }
           };
           auto issue_pv = [&](int t, int st, uint32_t acc) {
-            const uint32_t va = smem_u32(&s.v[st][0][0]);
+            const uint32_t b = vlo[st];
   #pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              mma_bf16_ts(tO[t], tS[t] + kk * 8, smem_desc_sw128(va + kk * 2048, kTileBytes, 1024), id_pv,
-                          (acc || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 8; ++kk)  // K-step of 16 keys: 8 TMEM columns of P, 2048 bytes of V
+              mma_bf16_ts_w(tO[t], tS[t] + kk * 8, b + kk * (2048 >> 4), dhi, id_pv, (acc || kk > 0) ? 1u : 0u);
           };
           bool ok = mbar_wait(&s.q_full[0], 0, abort_word, p.dc.err) &&
                     mbar_wait(&s.q_full[1], 0, abort_word, p.dc.err) &&
