@@ -31,6 +31,7 @@
 namespace vs {
 
 enum EstMode { kLse = 0, kSums = 1, kRecall = 2 };
+constexpr int kBinLevels = 16;  // recall levels binned in shared memory (the rest in registers)
 
 constexpr int kEstThreads = 384;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -64,7 +65,13 @@ struct __align__(1024) EstSmem {
   uint32_t tmem_base;
   int abort_word;
   float red[8][kRecallLevels];
+  // kRecall: per-thread bins of the first kBinLevels levels, [warpgroup][M tile of
+  // the thread][level][TMEM lane]; a thread owns its bins, and lane-major order puts
+  // a warp's 32 bins of one level in 32 distinct banks
+  float rbin[2][2][kBinLevels][kTile];
 };
+
+static_assert(sizeof(EstSmem) + 1024 <= 232448, "estimation shared memory exceeds 227 KB per CTA");
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -224,6 +231,12 @@ __global__ void __launch_bounds__(kEstThreads, 1)
       if (MODE != kLse && t < p.ntile && hh < p.g && r < p.nr)
         lse2[a] = p.lse[(G * p.g + hh) * kEstRows + r] * kLog2e;
     }
+    if (MODE == kRecall) {
+#pragma unroll
+      for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int l = 0; l < kBinLevels; ++l) s.rbin[wg][a][l][m] = 0.f;
+    }
     const int64_t irow = p.row0 + r;  // absolute position of this row
     bool ok = true;
     for (int i = 0; i < nb && ok; ++i) {
@@ -297,13 +310,16 @@ __global__ void __launch_bounds__(kEstThreads, 1)
               }
             } else {  // kRecall
               if (row_ok) {
-                // acc[t] is cumulative: it gathers A of the elements whose level is <= t.
-                // An element's level set is the bitmask ~0 << lv (levels t >= lv),
-                // restricted to the levels in use; masked-out (j > irow) elements have
+                // An element selected first at level lv (the smaller of its column's and
+                // its offset's level) belongs to every level t >= lv. Its probability goes
+                // to bin lv; the bins are prefix-summed over levels at the end. Levels at
+                // or above kBinLevels (only with tiny base budgets) are accumulated
+                // cumulatively in registers instead. Masked-out (j > irow) elements have
                 // v = 0 and read a clamped, in-range offset.
                 const uint8_t* lv_v = p.lvl + static_cast<int64_t>(h) * 2 * p.e_pad;
                 const uint8_t* lv_s = lv_v + p.e_pad;
-                const uint32_t levmask = (1u << p.nlev) - 1u;
+                const uint32_t nlev = static_cast<uint32_t>(p.nlev);
+                float* bins = &s.rbin[wg][a][0][m];
                 uint32_t vw[8];  // the 32 columns' vertical levels, 4 per word (same for all lanes)
 #pragma unroll
                 for (int q = 0; q < 8; ++q) vw[q] = __ldg(reinterpret_cast<const uint32_t*>(lv_v + j0) + q);
@@ -313,11 +329,14 @@ __global__ void __launch_bounds__(kEstThreads, 1)
                   const uint32_t lvv = (vw[x >> 2] >> (8 * (x & 3))) & 0xFFu;
                   const uint32_t lvs = __ldg(lv_s + (d >= 0 ? d : 0));
                   const uint32_t lv = lvv < lvs ? lvv : lvs;
-                  const uint32_t lm = lv < 32u ? ((0xFFFFFFFFu << lv) & levmask) : 0u;
+                  if (lv < nlev) {
+                    if (lv < static_cast<uint32_t>(kBinLevels)) {
+                      atomicAdd(bins + lv * kTile, v[x]);
+                    } else {
 #pragma unroll
-                  for (int t2 = 0; t2 < kRecallLevels; ++t2) {
-                    if (t2 >= p.nlev) break;  // uniform: levels in use only
-                    if ((lm >> t2) & 1u) acc[a][t2] += v[x];
+                      for (int t2 = kBinLevels; t2 < kRecallLevels; ++t2)
+                        if (static_cast<uint32_t>(t2) >= lv) acc[a][t2] += v[x];
+                    }
                   }
                 }
               }
@@ -339,6 +358,18 @@ __global__ void __launch_bounds__(kEstThreads, 1)
         }
       }
     } else if (MODE == kRecall) {
+      // this thread's bins (written by this thread only) as cumulative level sums
+#pragma unroll
+      for (int a = 0; a < 2; ++a) {
+        float run = 0.f;
+#pragma unroll
+        for (int l = 0; l < kBinLevels; ++l) {
+          run += s.rbin[wg][a][l][m];
+          acc[a][l] = run;
+        }
+#pragma unroll
+        for (int l = kBinLevels; l < kRecallLevels; ++l) acc[a][l] += run;
+      }
       // warp sums per level, then the two 32-row halves of each head in a fixed order
 #pragma unroll
       for (int a = 0; a < 2; ++a) {
