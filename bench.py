@@ -48,7 +48,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # taken on: a sha256 prefix over attn.cu, sm100.cuh and internal.cuh. A changed
 # kernel reports null until it is captured again.
 ATTN_TRAFFIC = {
-    "cfg2_qwen7b_n32k_refine": ("cbc89c1ab56f95f6", 665029376 + 199176704),
+    "cfg2_qwen7b_n32k_refine": ("d95398d87095c930", 602235136 + 201519104),
 }
 
 
