@@ -323,21 +323,44 @@ __global__ void __launch_bounds__(kEstThreads, 1)
                 uint32_t vw[8];  // the 32 columns' vertical levels, 4 per word (same for all lanes)
 #pragma unroll
                 for (int q = 0; q < 8; ++q) vw[q] = __ldg(reinterpret_cast<const uint32_t*>(lv_v + j0) + q);
+                auto bin_elements = [&](auto slash_level) {
 #pragma unroll
-                for (int x = 0; x < 32; ++x) {
-                  const int64_t d = irow - (j0 + x);
-                  const uint32_t lvv = (vw[x >> 2] >> (8 * (x & 3))) & 0xFFu;
-                  const uint32_t lvs = __ldg(lv_s + (d >= 0 ? d : 0));
-                  const uint32_t lv = lvv < lvs ? lvv : lvs;
-                  if (lv < nlev) {
-                    if (lv < static_cast<uint32_t>(kBinLevels)) {
-                      atomicAdd(bins + lv * kTile, v[x]);
-                    } else {
+                  for (int x = 0; x < 32; ++x) {
+                    const uint32_t lvv = (vw[x >> 2] >> (8 * (x & 3))) & 0xFFu;
+                    const uint32_t lvs = slash_level(x);
+                    const uint32_t lv = lvv < lvs ? lvv : lvs;
+                    if (lv < nlev) {
+                      if (lv < static_cast<uint32_t>(kBinLevels)) {
+                        atomicAdd(bins + lv * kTile, v[x]);
+                      } else {
 #pragma unroll
-                      for (int t2 = kBinLevels; t2 < kRecallLevels; ++t2)
-                        if (static_cast<uint32_t>(t2) >= lv) acc[a][t2] += v[x];
+                        for (int t2 = kBinLevels; t2 < kRecallLevels; ++t2)
+                          if (static_cast<uint32_t>(t2) >= lv) acc[a][t2] += v[x];
+                      }
                     }
                   }
+                };
+                // the offsets of this lane's 32 elements, irow - j0 - x, are the byte window
+                // [dbase, dbase + 31] of the slash levels, read backwards: eight or nine
+                // aligned words, funnel-shifted into place. Windows reaching below offset 0
+                // (the chunk at the diagonal) read byte by byte with the offset clamped.
+                const int64_t dbase = irow - j0 - 31;
+                if (dbase >= 0) {
+                  const uint32_t* wp = reinterpret_cast<const uint32_t*>(lv_s) + (dbase >> 2);
+                  const uint32_t sh = 8u * static_cast<uint32_t>(dbase & 3);
+                  uint32_t wv[9];
+#pragma unroll
+                  for (int q = 0; q < 8; ++q) wv[q] = __ldg(wp + q);
+                  wv[8] = sh ? __ldg(wp + 8) : 0u;  // the window's last byte is dbase + 31 <= irow < e_pad
+                  uint32_t aw[8];
+#pragma unroll
+                  for (int q = 0; q < 8; ++q) aw[q] = __funnelshift_r(wv[q], wv[q + 1], sh);
+                  bin_elements([&](int x) { return (aw[(31 - x) >> 2] >> (8 * ((31 - x) & 3))) & 0xFFu; });
+                } else {
+                  bin_elements([&](int x) {
+                    const int64_t d = irow - (j0 + x);
+                    return static_cast<uint32_t>(__ldg(lv_s + (d >= 0 ? d : 0)));
+                  });
                 }
               }
             }
