@@ -347,3 +347,108 @@ def layer_prefill(ctx: Context, q: torch.Tensor, k: torch.Tensor, v: torch.Tenso
             keep.append(dict(cs=cs, e=e, vert=vert, slash=slash, lse_est=lse, kv=kvb, ks=ksb, sets=sets,
                              recall=recall, lse=lse_o[:, cs:e], out=out[:, cs:e]))
     return out
+
+
+class HostStreamedPrefill:
+    """layer_prefill from pinned host memory, with the copies overlapped.
+
+    For a caller whose Q, K, V live in host memory and who wants O back there. The
+    work is cut into units of (chunk, KV-head group): no step of the path mixes KV
+    groups, and chunk c only needs the KV rows of chunks <= c. Each unit uploads its
+    new rows (the chunk's query rows of the group's heads, the chunk's K and V rows
+    of its KV heads) on an upload stream, computes estimate -> refine/select ->
+    sparse prefill on the caller's current stream with one library context per group,
+    and downloads its output rows on a download stream, so unit u's upload and unit
+    u-1's download run while unit u-1 computes. Results equal layer_prefill up to
+    rounding: a context over fewer KV heads splits the estimation's key range into
+    more parts, which changes the order of the partial sums.
+
+    Device buffers and contexts are allocated here, once; run() allocates nothing on
+    the device. kv_budget / ks_budget: ints or int32 [hq] tensors (e.g. calibrated)."""
+
+    def __init__(self, cfg: Config, seq_len: int, chunk: int, kv_budget, ks_budget, tau: Optional[float],
+                 max_iters: int = 19, kv_heads_per_unit: int = 1, device=None):
+        from dataclasses import replace
+
+        if cfg.hkv % kv_heads_per_unit:
+            raise ValueError("kv_heads_per_unit must divide hkv")
+        self.device = torch.device(device or "cuda")
+        dev = self.device
+        self.cfg, self.n, self.chunk, self.tau, self.max_iters = cfg, seq_len, chunk, tau, max_iters
+        g = cfg.hq // cfg.hkv
+        self.groups = [(k0, k0 + kv_heads_per_unit) for k0 in range(0, cfg.hkv, kv_heads_per_unit)]
+        hq_u = g * kv_heads_per_unit
+        self.ctxs = [Context(replace(cfg, hq=hq_u, hkv=kv_heads_per_unit), max_seq=seq_len,
+                             max_chunk=min(chunk, seq_len), device=dev) for _ in self.groups]
+        bf = torch.bfloat16
+        self.q = torch.empty(cfg.hq, seq_len, 128, dtype=bf, device=dev)
+        self.k = torch.empty(cfg.hkv, seq_len, 128, dtype=bf, device=dev)
+        self.v = torch.empty(cfg.hkv, seq_len, 128, dtype=bf, device=dev)
+        self.out = torch.empty_like(self.q)
+        self.lse = torch.empty(cfg.hq, seq_len, dtype=torch.float32, device=dev)
+
+        def per_head(b):
+            if isinstance(b, torch.Tensor):
+                return b.to(device=dev, dtype=torch.int32)
+            return torch.full((cfg.hq,), int(b), dtype=torch.int32, device=dev)
+
+        self.base_v, self.base_s = per_head(kv_budget), per_head(ks_budget)
+        f32, i32 = torch.float32, torch.int32
+        self.bufs = []
+        for _ in self.groups:
+            self.bufs.append(dict(
+                vert=torch.empty(hq_u, seq_len, dtype=f32, device=dev),
+                slash=torch.empty(hq_u, seq_len, dtype=f32, device=dev),
+                lse_est=torch.empty(hq_u, 64, dtype=f32, device=dev),
+                kv=torch.empty(hq_u, dtype=i32, device=dev), ks=torch.empty(hq_u, dtype=i32, device=dev),
+                recall=torch.empty(hq_u, dtype=f32, device=dev),
+                sets=(torch.empty(hq_u, seq_len, dtype=i32, device=dev), torch.empty(hq_u, dtype=i32, device=dev),
+                      torch.empty(hq_u, seq_len, dtype=i32, device=dev), torch.empty(hq_u, dtype=i32, device=dev))))
+        self.up = torch.cuda.Stream(device=dev)
+        self.down = torch.cuda.Stream(device=dev)
+        self.g = g
+
+    def run(self, q_h: torch.Tensor, k_h: torch.Tensor, v_h: torch.Tensor, out_h: torch.Tensor) -> None:
+        """q_h, out_h: [hq, N, 128]; k_h, v_h: [hkv, N, 128]; bf16, pinned host memory.
+        Asynchronous on the current stream: out_h is complete once it has synchronised."""
+        cfg, g = self.cfg, self.g
+        for t, shape in ((q_h, self.q.shape), (k_h, self.k.shape), (v_h, self.v.shape), (out_h, self.out.shape)):
+            if t.is_cuda or t.dtype != torch.bfloat16 or tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+                raise ValueError("host tensors must be contiguous bf16 [heads, N, 128] in host memory")
+        cur = torch.cuda.current_stream(self.device)
+        self.up.wait_stream(cur)    # the previous run's compute has read the device inputs
+        self.down.wait_stream(cur)
+        for ctx in self.ctxs:
+            ctx.reset()
+        for cs in range(0, self.n, self.chunk):
+            e = min(cs + self.chunk, self.n)
+            for ui, (k0, k1) in enumerate(self.groups):
+                h0, h1 = k0 * g, k1 * g
+                with torch.cuda.stream(self.up):
+                    for h in range(h0, h1):
+                        self.q[h, cs:e].copy_(q_h[h, cs:e], non_blocking=True)
+                    for h in range(k0, k1):
+                        self.k[h, cs:e].copy_(k_h[h, cs:e], non_blocking=True)
+                        self.v[h, cs:e].copy_(v_h[h, cs:e], non_blocking=True)
+                    ready = torch.cuda.Event()
+                    ready.record(self.up)
+                cur.wait_event(ready)
+                ctx, b = self.ctxs[ui], self.bufs[ui]
+                q, k, v = self.q[h0:h1], self.k[k0:k1], self.v[k0:k1]
+                vert, slash = b["vert"][:, :e], b["slash"][:, :e]
+                ctx.estimate(q, cs, k, e, out=(vert, slash, b["lse_est"]), full=True)
+                b["kv"].copy_(self.base_v[h0:h1])
+                b["ks"].copy_(self.base_s[h0:h1])
+                if self.tau is None:
+                    ctx.select(vert, slash, e, b["kv"], b["ks"], sets=b["sets"])
+                else:
+                    ctx.refine(q, cs, k, e, vert, slash, b["lse_est"], self.tau, b["kv"], b["ks"],
+                               max_iters=self.max_iters, sets=b["sets"], recall=b["recall"], full=True)
+                ctx.sparse_prefill(q, cs, e, k, v, b["sets"], out=self.out[h0:h1], lse=self.lse[h0:h1], full=True)
+                done = torch.cuda.Event()
+                done.record(cur)
+                with torch.cuda.stream(self.down):
+                    self.down.wait_event(done)
+                    for h in range(h0, h1):
+                        out_h[h, cs:e].copy_(self.out[h, cs:e], non_blocking=True)
+        cur.wait_stream(self.down)
