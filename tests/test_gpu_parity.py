@@ -11,7 +11,7 @@ import sparse_attention_estimate_b200 as vsb
 from sparse_attention_estimate_b200 import build as vsbuild
 from tests.gpu_common import (OUT_MAX_ABS, TAU_SLACK, assert_near_tie_equal, assert_outputs_close, f64,
                               layer_inputs, lists_to_sets, make_ctx, scale_of, sets_to_lists)
-from workloads import small_workload
+from workloads import generate_layer, small_workload
 
 pytestmark = pytest.mark.gpu
 
@@ -247,6 +247,39 @@ def test_sparse_prefill_matches_oracle(case, density):
             assert np.allclose(lse[h], ol, rtol=0, atol=2e-3), (name, density, cs, h, np.abs(lse[h] - ol).max())
         executed, useful = ctx.prefill_stats()
         assert executed > 0 and useful > 0
+
+
+@pytest.mark.parametrize("density", ["full", "mixed"])
+def test_sparse_prefill_with_large_jumps_of_the_row_max(density):
+    """Keys whose logits dwarf everything before them, in the first and in the second
+    64-key half of later 128-key blocks: the running row max of most query rows then
+    rises by far more than 2^16 (and exp2 against the old max overflows), which sends
+    the kernel's softmax through its redo-with-the-block's-own-max path and its O
+    rescale. Checked against the oracle like every other prefill."""
+    w = small_workload(2, seq_len=800, chunk=800, hq=2, hkv=1, n_planted=4)
+    lay = generate_layer(w)
+    spikes = [228, 276, 612, 670, 741]  # key offsets 100, 20, 100, 30, 101 inside their blocks
+    lay["k"][0, spikes] = (lay["k"][0, spikes].float() * 40.0).to(torch.bfloat16)
+    dev = {x: lay[x].cuda() for x in ("q", "k", "v")}
+    cpu = {x: f64(lay[x]) for x in ("q", "k", "v")}
+    ctx = make_ctx(w)
+    e = w.seq_len
+    if density == "full":
+        V, S = [np.arange(e, dtype=np.int64)] * w.hq, [np.array([0], np.int64)] * w.hq
+    else:
+        V, S = _random_sets(np.random.default_rng(11), w.hq, e, 0.3, 0.05)
+        V = [np.union1d(x, spikes).astype(np.int64) for x in V]
+    out, lse = ctx.sparse_prefill(dev["q"], 0, e, dev["k"], dev["v"], lists_to_sets(V, S, e, e))
+    assert ctx.status() == vsb.VS_OK
+    out, lse = f64(out), f64(lse)
+    rows = np.arange(e)
+    for h in range(w.hq):
+        oo, ol = vo.attention_rows(cpu["q"][h], rows, cpu["k"][0], cpu["v"][0], e, vo.membership(e, V[h]),
+                                   vo.membership(e, S[h]), w.rope_base, scale_of(w))
+        assert_outputs_close(out[h], oo, f"jumps {density} h={h}")
+        assert np.allclose(lse[h], ol, rtol=0, atol=2e-3), (density, h, np.abs(lse[h] - ol).max())
+    # the spikes do move the max: most rows past a spike attend mostly to it
+    assert np.max(np.abs(ol)) > 50.0
 
 
 def test_sparse_prefill_rows_without_keys_are_zero():
