@@ -71,3 +71,28 @@ def test_yarn_temperature():
     assert WORKLOADS[5].yarn_factor == 1.0 and WORKLOADS[5].softmax_scale == 1 / math.sqrt(128)
     short = small_workload(8, seq_len=1000, chunk=512, yarn_train_len=4096)
     assert short.yarn_factor == 1.0
+
+
+def test_planted_columns_stand_out_in_the_oracle_estimate():
+    """Workload sanity (not parity), on the 4096-token workload: the planted key columns
+    collect clearly more estimation mass than the other columns. Their boost is
+    K += 4u, Q += 1.5u, i.e. +6 raw, +0.53 scaled logits (x1.7 probability), which
+    puts every planted column above the median column but not all of them inside a
+    256-column budget: 8 of 16 make it on head 0 (the rest rank up to ~1500)."""
+    import numpy as np
+
+    import oracle.vs_oracle as vo
+    from workloads import WORKLOADS, generate_layer, structure
+
+    w = WORKLOADS[1]
+    planted = np.asarray(structure(w)["planted"])
+    lay = generate_layer(w)
+    q = lay["q"].float().double().numpy()
+    k = lay["k"].float().double().numpy()
+    e, nr = w.seq_len, w.last_q
+    others = np.setdiff1d(np.arange(e - 128), planted)  # outside the band of the estimation rows
+    for h in range(w.hq):
+        _, vert, _, _ = vo.estimate(q[h, e - nr:e], k[h // w.group], e, w.rope_base, w.softmax_scale)
+        assert vert[planted].mean() >= 2.0 * vert[others].mean(), h
+        rank = np.argsort(np.argsort(-vert, kind="stable"), kind="stable")
+        assert rank[planted].max() < e // 2, h
