@@ -357,6 +357,30 @@ class Layer:
             stats.append(ctx.prefill_stats())
 
 
+def job_workloads(args, rank: int, world: int):
+    """(this rank's workload, the job's workload, layers the job prefills): one layer's
+    KV groups over the ranks with --shard heads, else an independent layer per rank."""
+    if args.shard == "heads" and world > 1:
+        return shard_heads(select_workload(args), rank, world), select_workload(args), 1
+    w = rank_workload(select_workload(args), rank)
+    return (w, 0, 0), w, world
+
+
+def workload_config(args, w, wj, world: int, job_layers: int, cal_summary=None) -> dict:
+    """The JSON line's `config`: the workload, the same for both arms of the bench."""
+    return {
+        "workload": wj.name + ("_fullmask" if args.mask == "full" else ""), "seq_len": w.seq_len,
+        "hq": wj.hq, "hkv": wj.hkv, "head_dim": 128, "mask": args.mask, "q_scale": w.q_scale,
+        "softmax_scale": round(w.softmax_scale, 6),
+        "chunk": w.chunk, "n_chunks": w.n_chunks, "dca": [w.dca_chunk, w.dca_window] if w.dca_chunk else None,
+        "budgets": [w.kv_budget, w.ks_budget], "refine_tau": w.refine_tau,
+        "calibrated_budgets": cal_summary, "refine_positions": args.refine_positions,
+        "parallelism": ("single GPU" if world == 1 else f"KV groups of one layer over {world} GPUs"
+                        if job_layers == 1 else f"independent layer per GPU x{world}"),
+        "l2": "flushed between steps (256 MiB write)",
+    }
+
+
 def flush_l2(buf):
     buf.zero_()
 
@@ -367,18 +391,10 @@ def run_ours(args, rank, world, device):
 
     vsbuild.build()
     vsb.load_library()
-    if args.shard == "heads" and world > 1:  # one layer, KV groups over the ranks
-        w, q0, k0 = shard_heads(select_workload(args), rank, world)
-        lay = Layer(w, device, args.max_iters, full_mask=args.mask == "full", q0=q0, k0=k0,
-                    refine_dca=args.refine_positions == "dca")
-        lay.job_layers = 1
-        wj = select_workload(args)
-    else:  # an independent layer per rank
-        w = rank_workload(select_workload(args), rank)
-        lay = Layer(w, device, args.max_iters, full_mask=args.mask == "full",
-                    refine_dca=args.refine_positions == "dca")
-        lay.job_layers = world
-        wj = w
+    (w, q0, k0), wj, job_layers = job_workloads(args, rank, world)
+    lay = Layer(w, device, args.max_iters, full_mask=args.mask == "full", q0=q0, k0=k0,
+                refine_dca=args.refine_positions == "dca")
+    lay.job_layers = job_layers
     if args.calibrate:
         if w.refine_tau is None or args.mask == "full":
             raise SystemExit("--calibrate needs a workload with a refinement threshold and --mask selected")
@@ -450,17 +466,7 @@ def run_ours(args, rank, world, device):
         "dtype": "bf16",
         "data": ("synthetic (seeded generator: N(0,1) Q/K/V" + (f", Q's N(0,1) part x{w.q_scale:g}" if w.q_scale != 1
                  else "") + ", planted verticals, 64-aligned band)"),
-        "config": {
-            "workload": wj.name + ("_fullmask" if args.mask == "full" else ""), "seq_len": w.seq_len,
-            "hq": wj.hq, "hkv": wj.hkv, "head_dim": 128, "mask": args.mask, "q_scale": w.q_scale,
-            "softmax_scale": round(w.softmax_scale, 6),
-            "chunk": w.chunk, "n_chunks": nchunks, "dca": [w.dca_chunk, w.dca_window] if w.dca_chunk else None,
-            "budgets": [w.kv_budget, w.ks_budget], "refine_tau": w.refine_tau,
-            "calibrated_budgets": lay.cal_summary, "refine_positions": args.refine_positions,
-            "parallelism": ("single GPU" if world == 1 else f"KV groups of one layer over {world} GPUs"
-                            if lay.job_layers == 1 else f"independent layer per GPU x{world}"),
-            "l2": "flushed between steps (256 MiB write)",
-        },
+        "config": workload_config(args, w, wj, world, lay.job_layers, lay.cal_summary),
         "executed_tflops": round(exec_flops / (ms_per_step / 1e3) / 1e12, 2),
         "attn_executed_tflops": round(attn_tflops, 2),
         "pct_bf16_peak": round(100 * attn_tflops / peak, 2),
@@ -608,8 +614,9 @@ def cpu_cores():
         return os.cpu_count()
 
 
-def run_reference(args):
+def run_reference(args, world: int = 1):
     w = select_workload(args)
+    (wr, _, _), wj, job_layers = job_workloads(args, 0, world)
     for _ in range(args.warmup):
         oracle_sample(w, budget_s=2.0, n_rows=16, seed=99)
     vals = []
@@ -623,7 +630,7 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(w.seq_len / value * 1e3, 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded generator)",
-        "config": {"workload": w.name, "seq_len": w.seq_len, "hq": w.hq, "hkv": w.hkv},
+        "config": workload_config(args, wr, wj, world, job_layers),
         "cpu_baseline": cb,
         "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -638,7 +645,7 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         if rank == 0:
-            print(json.dumps(run_reference(args)), flush=True)
+            print(json.dumps(run_reference(args, world)), flush=True)
         return 0
     if not torch.cuda.is_available():
         print(json.dumps({"metric": METRIC, "error": "no CUDA device"}))
