@@ -79,3 +79,14 @@ def test_calls_reject_null_context(lib):
                                  None) == vsb.VS_ERR_INVALID_ARG
     assert lib.vs_context_reset(None) == vsb.VS_ERR_INVALID_ARG
     assert lib.vs_set_wait_limit(None, 10 ** 9) == vsb.VS_ERR_INVALID_ARG
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="checks the behaviour without a CUDA device")
+def test_python_entry_points_fail_loudly_without_a_gpu():
+    """No CPU fallback: without a CUDA device every entry point of the binding raises
+    before doing any work (the oracle is test infrastructure, never a product path)."""
+    cfg = vsb.Config(hq=2, hkv=1)
+    with pytest.raises(RuntimeError, match="CUDA"):
+        vsb.Context(cfg, max_seq=256, max_chunk=256)
+    with pytest.raises(RuntimeError, match="CUDA"):
+        vsb.HostStreamedPrefill(cfg, 256, 256, 8, 8, None)
