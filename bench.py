@@ -43,6 +43,10 @@ from workloads import WORKLOADS, generate_head, structure  # noqa: E402
 METRIC = "sparse-prefill tokens/s per layer; executed TFLOP/s and % of B200 BF16 peak"
 FLOP_PER_TILE = 4 * 128 * 128 * 128  # QK^T and PV of one executed 128-query x 128-key tile
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# NVIDIA's published dense BF16 tensor figure for one B200 (the 4.5 PFLOP/s of the
+# datasheet is with 2:4 sparsity); reported beside the measured peaks, never as the
+# roofline denominator.
+DATASHEET_BF16_TFLOPS = 2250.0
 # DRAM bytes (read + write) of one attention-kernel launch, from one ncu capture per
 # workload (the attention-kernel summaries under profiles/), valid only for the kernel sources they were
 # taken on: a sha256 prefix over attn.cu, sm100.cuh and internal.cuh. A changed
@@ -75,7 +79,8 @@ def parse():
     p.add_argument("--steps", type=int, default=5)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--config", type=int, default=2, choices=sorted(WORKLOADS))
+    p.add_argument("--config", type=int, default=5, choices=sorted(WORKLOADS),
+                   help="workload (default 5: 40/8 heads, 1M tokens in 32 chunks, DCA 262144, refinement 0.9)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--max-iters", type=int, default=19)
@@ -471,6 +476,7 @@ def run_ours(args, rank, world, device):
         "attn_executed_tflops": round(attn_tflops, 2),
         "pct_bf16_peak": round(100 * attn_tflops / peak, 2),
         "pct_bf16_peak_of": f"{pk_src} {'sustained' if long_step else 'burst'} {peak} TFLOP/s",
+        "pct_bf16_datasheet_peak": round(100 * attn_tflops / DATASHEET_BF16_TFLOPS, 2),
         "useful_tflops": round(useful_flops / (ms_per_step / 1e3) / 1e12, 2),
         "density_useful_over_executed": round(useful_flops / exec_flops, 4) if exec_flops else None,
         "attn_ms_per_step": round(attn_ms_step, 3),
@@ -487,15 +493,18 @@ def run_ours(args, rank, world, device):
     }
     # ---------------------------------------------------------------- end to end (host buffers)
     if not args.no_e2e:
-        res["e2e"] = run_e2e(args, lay, l2, world, device)
+        res["e2e"] = run_e2e(args, lay, l2, world, device, ms_per_step)
     return res, w, lay
 
 
-def run_e2e(args, lay, l2, world, device):
+def run_e2e(args, lay, l2, world, device, ms_per_step):
     """Same step through the public API from pinned host memory: H2D of q, k, v
     and D2H of the output inside the timed region. With the selected mask the step
-    is HostStreamedPrefill (uploads, compute and downloads of (chunk, KV head) units
-    overlapped on three streams); with --mask full, copies then the step."""
+    is HostStreamedPrefill (uploads, compute and downloads of work units overlapped
+    on three streams): units of (chunk, KV head) for a single-chunk layer, whole
+    chunks otherwise (each chunk's attention then fills the GPU in one launch);
+    with --mask full, copies then the step. Seconds-long steps time fewer e2e steps
+    (about 40 s in all, at least 2); the line gives the count."""
     hq_h = lay.q.cpu().pin_memory()
     hk_h = lay.k.cpu().pin_memory()
     hv_h = lay.v.cpu().pin_memory()
@@ -503,9 +512,11 @@ def run_e2e(args, lay, l2, world, device):
     w = lay.w
     if not lay.full_mask:
         tau = None if (w.refine_tau is None or lay.calibrated) else w.refine_tau
+        per_unit = 1 if w.n_chunks == 1 else w.hkv
         sp = lay.vsb.HostStreamedPrefill(lay.ctx.cfg, w.seq_len, w.chunk, lay.base_v, lay.base_s, tau,
-                                         max_iters=lay.max_iters, device=device)
-        mode = "streamed: (chunk, KV head) units, uploads and downloads overlapped with compute"
+                                         max_iters=lay.max_iters, kv_heads_per_unit=per_unit, device=device)
+        mode = ("streamed: (chunk, KV head) units" if per_unit == 1 else "streamed: chunk units") + \
+            ", uploads and downloads overlapped with compute"
 
         def e2e_step():
             sp.run(hq_h, hk_h, hv_h, out_h)
@@ -520,13 +531,15 @@ def run_e2e(args, lay, l2, world, device):
             lay.step(q=dq, k=dk, v=dv)
             out_h.copy_(lay.out, non_blocking=True)
 
-    for _ in range(2):
+    long_step = ms_per_step > 2000.0
+    n_steps = max(2, min(args.steps, int(40000.0 // max(ms_per_step, 1e-3))))
+    for _ in range(1 if long_step else 2):
         e2e_step()
     torch.cuda.synchronize()
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_steps)]
     if world > 1:
         torch.distributed.barrier()
-    for i in range(args.steps):
+    for i in range(n_steps):
         flush_l2(l2)
         evs[i][0].record()
         e2e_step()
@@ -535,9 +548,9 @@ def run_e2e(args, lay, l2, world, device):
     tot = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), world, device)
     h2d = (hq_h.numel() + hk_h.numel() + hv_h.numel()) * 2
     d2h = out_h.numel() * 2
-    return {"value": round(job_throughput(lay.w.seq_len, args.steps, lay.job_layers, tot), 1), "unit": "tokens/s",
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(tot / args.steps, 3),
-            "mode": mode}
+    return {"value": round(job_throughput(lay.w.seq_len, n_steps, lay.job_layers, tot), 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(tot / n_steps, 3),
+            "steps": n_steps, "mode": mode}
 
 
 # ----------------------------------------------------------------------------- the CPU oracle
@@ -545,26 +558,35 @@ def oracle_sample(w, budget_s=15.0, n_rows=64, seed=0):
     """Times the oracle on a bounded sample of workload w and extrapolates to the
     layer. Work units are (head, chunk) pairs: the chunk's estimation, selection
     and refinement for that head, plus the attention of n_rows sampled query rows
-    of the chunk. Units run in a spread order (heads in turn, chunks from the
-    last, longest one down) until budget_s of wall time is spent (at least one
-    unit). Each unit's cost is taken as linear in its key count e (estimation and
-    per-row attention both are), so the measured per-key rates extrapolate to
-    every chunk, row and head. Returns (tokens/s, seconds spent, description)."""
+    of the chunk. Chunks are taken from a spread over the sequence (first, last and
+    up to three between), smallest first, heads in turn; a unit whose predicted
+    cost (the per-key rates measured so far times its key count) exceeds the time
+    left is skipped, so one sample stays near budget_s even where one unit at the
+    longest chunk would take longer. Each unit's cost is taken as linear in its key
+    count e (estimation and per-row attention both are), so the measured per-key
+    rates extrapolate to every chunk, row and head. Returns (tokens/s, seconds
+    spent, description)."""
     import oracle.vs_oracle as vo
 
     st = structure(w)
     rng = np.random.default_rng(seed)
     dca = (w.dca_chunk, w.dca_window) if w.dca_chunk else None
     scale = w.softmax_scale
-    chunks = list(range(w.n_chunks - 1, -1, -1))
-    units = [(h, c) for c in chunks for h in range(w.hq)]
+    spread = sorted(set(int(round(x)) for x in np.linspace(0, w.n_chunks - 1, min(w.n_chunks, 5))))
+    units = [((r * len(spread) + i) % w.hq, c) for r in range(w.hq) for i, c in enumerate(spread)]
     fixed_per_key, row_per_key = [], []  # seconds per key of e: per chunk, and per row and chunk
-    cache = {}
-    spent0 = time.time()
-    done = 0
+    cache = _ORACLE_INPUTS.setdefault(w, {})  # generated heads, kept across samples
+    spent = 0.0  # oracle time only: generating the inputs is not part of the sample
+    wall0 = time.time()
+    done, chunks_seen = 0, set()
     for h, c in units:
-        if done and time.time() - spent0 >= budget_s:
+        left = budget_s - spent
+        if done and (left <= 0 or time.time() - wall0 > 4 * budget_s):
             break
+        cs, e = w.chunk_bounds(c)
+        nrow = min(n_rows, e - cs)
+        if done and (np.mean(fixed_per_key) + nrow * np.mean(row_per_key)) * e > left:
+            continue  # predicted to overrun the budget
         hk = h // w.group
         if ("k", hk) not in cache:
             cache = {k: v for k, v in cache.items() if k[0] != "k" and k[0] != "v"}
@@ -574,7 +596,6 @@ def oracle_sample(w, budget_s=15.0, n_rows=64, seed=0):
             cache = {k: v for k, v in cache.items() if k[0] != "q"}
             cache[("q", h)] = generate_head(w, "q", h, st=st).float().double().numpy()
         kf, vf, qf = cache[("k", hk)], cache[("v", hk)], cache[("q", h)]
-        cs, e = w.chunk_bounds(c)
         nr = min(w.last_q, e - cs)
         t0 = time.time()
         _, vert, slash, a = vo.estimate(qf[e - nr : e], kf, e, w.rope_base, scale)
@@ -584,7 +605,7 @@ def oracle_sample(w, budget_s=15.0, n_rows=64, seed=0):
             _, _, V, S, _, _ = vo.refine(a, np.arange(e - nr, e), vert, slash, w.kv_budget, w.ks_budget,
                                          w.refine_tau)
         t1 = time.time()
-        rows = np.sort(rng.choice(np.arange(cs, e), size=min(n_rows, e - cs), replace=False))
+        rows = np.sort(rng.choice(np.arange(cs, e), size=nrow, replace=False))
         inV, inS = vo.membership(e, V), vo.membership(e, S)
         # two-point fit: one row (the call's fixed cost, e.g. rotating the keys) and all rows
         vo.attention_rows(qf[rows[-1:]], rows[-1:], kf, vf, e, inV, inS, w.rope_base, scale, dca)
@@ -595,16 +616,21 @@ def oracle_sample(w, budget_s=15.0, n_rows=64, seed=0):
         fixed = max((t2 - t1) - per_row, 0.0)
         fixed_per_key.append(((t1 - t0) + fixed) / e)
         row_per_key.append(per_row / e)
+        spent += t3 - t0
         done += 1
+        chunks_seen.add(c)
     fk, rk = float(np.mean(fixed_per_key)), float(np.mean(row_per_key))
     layer_s = 0.0
     for c in range(w.n_chunks):
         cs, e = w.chunk_bounds(c)
         layer_s += w.hq * (fk * e + rk * e * (e - cs))
-    desc = (f"{done} of {len(units)} (head, chunk) units, each the chunk's estimation+selection"
-            f"{'+refinement' if w.refine_tau else ''} for one head and {n_rows} sampled query rows of its "
-            f"attention; per-key rates extrapolated to every row, chunk and head")
-    return w.seq_len / layer_s, time.time() - spent0, desc
+    desc = (f"{done} (head, chunk) units of {w.hq * w.n_chunks} (chunks {sorted(chunks_seen)}), each the chunk's "
+            f"estimation+selection{'+refinement' if w.refine_tau else ''} for one head and up to {n_rows} sampled "
+            f"query rows of its attention; per-key rates extrapolated to every row, chunk and head")
+    return w.seq_len / layer_s, spent, desc
+
+
+_ORACLE_INPUTS: dict = {}
 
 
 def cpu_cores():
@@ -619,15 +645,18 @@ def run_reference(args, world: int = 1):
     (wr, _, _), wj, job_layers = job_workloads(args, 0, world)
     for _ in range(args.warmup):
         oracle_sample(w, budget_s=2.0, n_rows=16, seed=99)
-    vals = []
+    vals, walls = [], []
     for i in range(args.steps):
         v, spent, desc = oracle_sample(w, budget_s=8.0, n_rows=32, seed=i)
         vals.append(v)
+        walls.append(spent)
     value = statistics.median(vals)
     cb = {"value": round(value, 3), "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle", "sample": desc}
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(w.seq_len / value * 1e3, 1),
+        # a step is a bounded sample: ms_per_step is the layer time extrapolated from it
+        "extrapolated": True, "timed_wall_s_per_step": round(statistics.mean(walls), 2),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded generator)",
         "config": workload_config(args, wr, wj, world, job_layers),

@@ -196,8 +196,10 @@ VS_API vs_status vs_set_prefill_events(vs_ctx* ctx, cudaEvent_t start, cudaEvent
  * of 32 MiB per device, held by every GPU that loads the library until exit;
  * hq * 2 * round_up(e, 128) bytes plus ~hq * 512 bytes must fit, else
  * VS_ERR_UNSUPPORTED. Nothing is allocated. The first call on a device looks up
- * the array's device address (make it before any stream capture begins). Calls
- * on one device share the array: calls whose kernels overlap on the GPU race.
+ * the array's device address (make it before any stream capture begins); the
+ * lookup is repeated when another CUDA context is current on that device, e.g.
+ * after cudaDeviceReset. Calls on one device share the array: calls whose
+ * kernels overlap on the GPU race.
  */
 VS_API vs_status vs_select_noalloc(int32_t hq, const float* vert, const float* slash,
                                    int64_t e_ld, int64_t e, const int32_t* kv_budget,

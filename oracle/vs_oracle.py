@@ -105,19 +105,23 @@ def dca_positions(i: int, j, C: int, W: int):
 
 
 # ----------------------------------------------------------------------------- estimation  [QW Sparse Attention, Chunked Prefill]
-def estimate(q_rows: np.ndarray, k: np.ndarray, e: int, base: float, scale: float):
+def estimate(q_rows: np.ndarray, k: np.ndarray, e: int, base: float, scale: float,
+             k_rot: Optional[np.ndarray] = None):
     """Attention of the chunk's last queries against every visible key, with
     continuous positions ([QW] "Algorithm": select with continuous positions;
     "Chunked Prefill": the last 64 queries of each chunk).
 
     q_rows: (nr x d) pre-RoPE queries at positions e-nr .. e-1; k: (>= e x d)
     pre-RoPE keys of the matching KV head. Causal: query i sees keys j <= i.
+    k_rot: optionally rope(k, arange, base) already computed (rows >= e), so that
+    a caller estimating many chunks of one KV head rotates its keys once; the
+    same rows, the same arithmetic.
     Returns lse (nr,), vert (e,) with vert[j] = sum_i A_ij, and slash (e,) with
     slash[dd] = sum_i A_{i, i-dd}, where A = row softmax of the scaled scores."""
     nr = q_rows.shape[0]
     rows = np.arange(e - nr, e)
     qr = rope(q_rows, rows, base)
-    kr = rope(k[:e], np.arange(e), base)
+    kr = rope(k[:e], np.arange(e), base) if k_rot is None else k_rot[:e]
     s = scale * (qr @ kr.T)
     cols = np.arange(e)
     s = np.where(cols[None, :] <= rows[:, None], s, _NEG_INF)
@@ -156,30 +160,54 @@ def estimate_probs_dca(q_rows: np.ndarray, k: np.ndarray, e: int, base: float, s
 
 
 # ----------------------------------------------------------------------------- selection  [QW Sparse Attention]
-def topk_sorted(score: np.ndarray, k: int) -> np.ndarray:
+def ranking(score: np.ndarray) -> np.ndarray:
+    """All indices ranked by (score descending, index ascending)."""
+    n = score.shape[0]
+    return np.lexsort((np.arange(n), -score))
+
+
+def topk_sorted(score: np.ndarray, k: int, order: Optional[np.ndarray] = None) -> np.ndarray:
     """Indices of the k largest scores, ranked by (score descending, index
-    ascending), returned in ascending index order."""
+    ascending), returned in ascending index order. order: ranking(score) when
+    the caller has it already (the same ranking, computed once)."""
     n = score.shape[0]
     k = min(int(k), n)
-    order = np.lexsort((np.arange(n), -score))
+    if order is None:
+        order = ranking(score)
     return np.sort(order[:k]).astype(np.int64)
 
 
-def kth_score(score: np.ndarray, k: int) -> float:
+def kth_score(score: np.ndarray, k: int, order: Optional[np.ndarray] = None) -> float:
+    """The score of the k-th ranked element (k capped at the length): the
+    boundary of the top-k set."""
     n = score.shape[0]
     k = min(int(k), n)
-    order = np.lexsort((np.arange(n), -score))
+    if order is None:
+        order = ranking(score)
     return float(score[order[k - 1]])
 
 
-def select(vert: np.ndarray, slash: np.ndarray, kv: int, ks: int):
+def slash_scores(slash: np.ndarray) -> np.ndarray:
+    """The slash scores as ranked by the selection: offset 0 (the main
+    diagonal) forced in front of every other offset."""
+    sl = slash.copy()
+    sl[0] = np.inf
+    return sl
+
+
+def select_orders(vert: np.ndarray, slash: np.ndarray):
+    """(ranking of vert, ranking of the slash scores with offset 0 forced)."""
+    return ranking(vert), ranking(slash_scores(slash))
+
+
+def select(vert: np.ndarray, slash: np.ndarray, kv: int, ks: int, orders=None):
     """Critical tokens of the vertical-slash pattern ([QW] Sparse Attention, step
     3): the kv columns with the largest vertical scores and the ks diagonal
     offsets with the largest slash scores. Offset 0 (the main diagonal) is
-    always selected. Both lists ascending."""
-    sl = slash.copy()
-    sl[0] = np.inf
-    return topk_sorted(vert, kv), topk_sorted(sl, ks)
+    always selected. Both lists ascending. orders: select_orders(vert, slash)
+    when the caller has them already."""
+    ov, osl = orders if orders is not None else (None, None)
+    return topk_sorted(vert, kv, ov), topk_sorted(slash_scores(slash), ks, osl)
 
 
 def membership(e: int, idx: np.ndarray) -> np.ndarray:
@@ -192,12 +220,13 @@ def recall(a: np.ndarray, rows: np.ndarray, inV: np.ndarray, inS: np.ndarray) ->
     """Attention recall of the estimation rows ([QW] Sparsity Refinement):
     per row, exp(lse_sparse - lse_full) = sum of A_ij over the selected keys;
     the head's recall is the mean over the rows."""
-    e = a.shape[1]
-    j = np.arange(e)
     tot = 0.0
     for r, i in enumerate(rows):
-        sel = (j <= i) & (inV | inS[np.clip(i - j, 0, e - 1)])
-        tot += a[r, sel].sum()
+        i = int(i)
+        # keys j = 0 .. i: column j selected, or offset i - j selected (inS read backwards
+        # from offset i down to offset 0)
+        sel = inV[: i + 1] | inS[i::-1]
+        tot += a[r, : i + 1][sel].sum()
     return tot / len(rows)
 
 
@@ -210,8 +239,9 @@ def refine(a: np.ndarray, rows: np.ndarray, vert: np.ndarray, slash: np.ndarray,
     e = vert.shape[0]
     kv, ks = min(int(kv), e), min(int(ks), e)
     trace = []
+    orders = select_orders(vert, slash)  # the ranking does not change between steps
     for it in range(max_iters + 1):
-        V, S = select(vert, slash, kv, ks)
+        V, S = select(vert, slash, kv, ks, orders)
         rc = recall(a, rows, membership(e, V), membership(e, S))
         trace.append((kv, ks, rc))
         if rc >= tau or (kv >= e and ks >= e) or it == max_iters:
@@ -260,12 +290,15 @@ def attention_rows_dense(q_rows: np.ndarray, rows: np.ndarray, k: np.ndarray, v:
 
 def attention_rows(q_rows: np.ndarray, rows: np.ndarray, k: np.ndarray, v: np.ndarray, e: int,
                    inV: np.ndarray, inS: np.ndarray, base: float, scale: float,
-                   dca: Optional[tuple] = None, block: int = 128):
+                   dca: Optional[tuple] = None, block: int = 128, k_rot: Optional[np.ndarray] = None,
+                   round_out: bool = True):
     """Same arithmetic as `attention_rows_dense`, evaluated for blocks of rows at
     a time over the keys the block can see (masked entries are -inf and
-    contribute exactly zero)."""
+    contribute exactly zero). k_rot: optionally the keys already rotated to their
+    key positions (rope(k, _key_positions(n, dca), base), rows >= e). round_out:
+    False returns the float64 outputs before their final rounding to bf16."""
     rows = np.asarray(rows, dtype=np.int64)
-    kr = rope(k[:e], _key_positions(e, dca), base)
+    kr = rope(k[:e], _key_positions(e, dca), base) if k_rot is None else k_rot[:e]
     out = np.zeros((len(rows), v.shape[1]))
     lse = np.zeros(len(rows))
     for b0 in range(0, len(rows), block):
@@ -293,7 +326,13 @@ def attention_rows(q_rows: np.ndarray, rows: np.ndarray, k: np.ndarray, v: np.nd
         den = w.sum(axis=1, keepdims=True)
         lse[b0 : b0 + block] = (mx + np.log(den))[:, 0]
         out[b0 : b0 + block] = (w / den) @ v[:hi]
-    return bf16_rne(out), lse
+    return (bf16_rne(out) if round_out else out), lse
+
+
+def key_positions(e: int, dca: Optional[tuple] = None) -> np.ndarray:
+    """Positions the keys 0 .. e-1 are rotated to in attention: j, or j mod (C - W)
+    under DCA ([QW] Length Extrapolation)."""
+    return _key_positions(e, dca)
 
 
 # ----------------------------------------------------------------------------- the chunk loop  [QW Algorithm; Chunked Prefill]
@@ -325,7 +364,7 @@ def calibrate(q: np.ndarray, k: np.ndarray, *, chunk: int, last_q: int, kv_budge
 def layer_prefill(q: np.ndarray, k: np.ndarray, v: np.ndarray, *, chunk: int, last_q: int,
                   kv_budget, ks_budget, tau: Optional[float], base: float,
                   scale: Optional[float] = None, dca: Optional[tuple] = None,
-                  rows_per_chunk=None, max_iters: int = 64, heads=None):
+                  rows_per_chunk=None, max_iters: int = 64, heads=None, round_out: bool = True):
     """One attention layer's chunked prefill ([QW] "Algorithm"): for each chunk
     [cs, e) of `chunk` queries over the keys [0, e), select the critical tokens
     per head from the chunk's last `last_q` queries with continuous positions,
@@ -336,7 +375,8 @@ def layer_prefill(q: np.ndarray, k: np.ndarray, v: np.ndarray, *, chunk: int, la
     kv_budget / ks_budget: one int for every head, or a sequence with one budget
     per head (calibrated budgets, used with tau None).
     rows_per_chunk: None (every row) or a function (cs, e) -> absolute rows to
-    evaluate. Returns a list with one dict per chunk."""
+    evaluate. round_out: False keeps the outputs in float64 (before the final
+    bf16 rounding). Returns a list with one dict per chunk."""
     hq, n, d = q.shape
     hkv = k.shape[0]
     g = hq // hkv
@@ -363,7 +403,7 @@ def layer_prefill(q: np.ndarray, k: np.ndarray, v: np.ndarray, *, chunk: int, la
             else:
                 kv, ks, V, S, rc, trace = refine(a, est_rows, vert, slash, kvb, ksb, tau, max_iters)
             o, lse = attention_rows(q[h, rows], rows, kh, vh, e, membership(e, V), membership(e, S),
-                                    base, scale, dca)
+                                    base, scale, dca, round_out=round_out)
             per[h] = dict(lse_est=lse_e, vert=vert, slash=slash, kv=kv, ks=ks, V=V, S=S,
                           recall=rc, trace=trace, rows=rows, out=o, lse=lse)
         res.append(dict(cs=cs, e=e, heads=per))

@@ -249,10 +249,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   AttnSmem& s = *reinterpret_cast<AttnSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // longest work first: pairs in descending order, the heads of a KV group adjacent
-  const int pair = p.npairs - 1 - static_cast<int>(blockIdx.x / p.hq);
-  const int h = static_cast<int>(blockIdx.x % p.hq);
-  const int hk = h / p.g;
+  // Work order: the KV groups one after another; inside a group the query-tile pairs
+  // longest first, the g heads of a pair adjacent. The CTAs resident at any time then
+  // belong to one KV head (two at a group boundary) and start together, so they sweep
+  // its K/V blocks nearly in step and share each block through L2; with the heads of
+  // all groups interleaved, a chunk's K/V (up to 4.3 GB at 1M keys) was re-read from HBM.
+  const int per_group = p.npairs * p.g;
+  const int hk = static_cast<int>(blockIdx.x) / per_group;
+  const int rg = static_cast<int>(blockIdx.x) % per_group;
+  const int pair = p.npairs - 1 - rg / p.g;
+  const int h = hk * p.g + rg % p.g;
   const int64_t R0 = p.q_pos0 + static_cast<int64_t>(pair) * 256;  // tile 0's first row
   const int32_t* list = p.sched + (static_cast<int64_t>(h) * p.npairs_ws + pair) * p.nblk_ws;
   const int n = p.sched_cnt[static_cast<int64_t>(h) * p.npairs_ws + pair];

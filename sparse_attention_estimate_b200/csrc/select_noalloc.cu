@@ -14,12 +14,17 @@
 // when the library's device code is loaded; with CUDA's lazy module loading
 // that happens at the first call here). Its host-side name is only a
 // stand-in, so its device address is fetched with cudaGetSymbolAddress, once
-// per device, the first time this entry point runs with that device current
-// (make that first call before any stream capture begins). All calls
-// share the array and it keeps the last call's contents; the kernels overwrite
-// every byte they read, so nothing needs clearing, but two calls on one device
-// whose kernels overlap on the GPU (for example on two streams) race on it:
-// serialise them. Each device has its own copy of the array.
+// per device and CUDA context, the first time this entry point runs with that
+// device current (make that first call before any stream capture begins). The
+// address is cached against the context that was current at the lookup: after
+// a cudaDeviceReset, or under another context on the same device, the module is
+// loaded again at another address, and the next call looks it up again. All
+// calls share the array and it keeps the last call's contents; the kernels
+// overwrite every byte they read, so nothing needs clearing, but two calls on
+// one device whose kernels overlap on the GPU (for example on two streams) race
+// on it: serialise them. Each device has its own copy of the array.
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "internal.cuh"
@@ -36,21 +41,55 @@ vs_status launch_select_raw(int hq, const float* vert, const float* slash, int64
                             int64_t e_pad, int* err, int32_t* v_idx, int32_t cap_v, int32_t* v_cnt,
                             int32_t* s_off, int32_t cap_s, int32_t* s_cnt, cudaStream_t st);
 
-// Device address of the scratch array on the current device (looked up once).
+// Driver calls through the runtime's driver entry point (no link against libcuda).
+template <class Fn>
+static Fn driver_fn(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) == cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    return reinterpret_cast<Fn>(p);
+  return nullptr;
+}
+
+// Process-unique id of the current context (0 when none is current). Context ids
+// are never reused within a process, unlike context handles.
+static unsigned long long current_context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_ctx = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    get_ctx = driver_fn<PFN_cuCtxGetCurrent_v4000>("cuCtxGetCurrent");
+    get_id = driver_fn<PFN_cuCtxGetId_v12000>("cuCtxGetId");
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_ctx || !get_id || get_ctx(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of the scratch array on the current device. The lookup (which
+// also initialises the device's context and loads the module on first use) runs
+// once per device and context: again whenever the current context is not the one
+// of the cached lookup, e.g. after cudaDeviceReset.
 static vs_status scratch_address(unsigned char** out) {
   static std::mutex mu;
   static unsigned char* addr[kNoAllocMaxDevices] = {};
+  static unsigned long long owner[kNoAllocMaxDevices] = {};
   int dev = -1;
   vs_status s = cuda_check(cudaGetDevice(&dev), "cudaGetDevice");
   if (s != VS_OK) return s;
   if (dev < 0 || dev >= kNoAllocMaxDevices)
     return set_error(VS_ERR_UNSUPPORTED, "device ordinal %d beyond %d", dev, kNoAllocMaxDevices);
   std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
+  const unsigned long long id = current_context_id();
+  if (!addr[dev] || id == 0 || owner[dev] != id) {
     void* p = nullptr;
     s = cuda_check(cudaGetSymbolAddress(&p, g_select_scratch), "cudaGetSymbolAddress(scratch)");
     if (s != VS_OK) return s;
     addr[dev] = static_cast<unsigned char*>(p);
+    owner[dev] = current_context_id();  // the context the lookup ran in
   }
   *out = addr[dev];
   return VS_OK;

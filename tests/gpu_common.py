@@ -70,18 +70,41 @@ def assert_near_tie_equal(got, want, score, k):
         assert abs(s - kth) <= tol or (np.isinf(s) and np.isinf(kth)), (j, s, kth)
 
 
-def assert_outputs_close(got: np.ndarray, want: np.ndarray, what="", w=None):
-    """Spec bounds: max abs 2e-2, mean abs 2e-3. For the sparse-regime workloads
-    (q_scale != 1) attention concentrates on few keys, so outputs reach the size of
-    single V rows (|O| up to ~4) and both sides' bf16 rounding of O can land one
-    output ulp apart: there each element may also differ by one bf16 ulp of the
-    oracle's value (ulp(x) <= 2^-7 |x|), and the mean by half of that on average."""
-    d = np.abs(got - want)
+def bf16_half_ulp(x: np.ndarray) -> np.ndarray:
+    """Half the spacing of bfloat16 values (8 significant bits) at |x|: the largest
+    error of one correct rounding of x to bf16."""
+    a = np.abs(x)
+    ex = np.floor(np.log2(np.maximum(a, 2.0 ** -126)))
+    return np.where(a > 0, np.exp2(ex - 8), 0.0)
+
+
+def assert_outputs_close(got: np.ndarray, exact: np.ndarray, what="", w=None):
+    """GPU bf16 outputs against the oracle's float64 outputs before their final
+    rounding (oracle attention with round_out=False).
+
+    Spec bounds: max abs 2e-2 and mean abs 2e-3 against the oracle's bf16
+    output. For the sparse-regime workloads (q_scale != 1) attention concentrates
+    on few keys and outputs reach the size of single V rows (|O| up to ~4), where
+    two correct bf16 roundings of nearly equal values can land one bf16 step apart
+    (0.031 at |O| in [4, 8)). There the GPU output is compared with the exact value
+    instead, allowing the bounds plus half a bf16 step at that value: the GPU's own
+    rounding of its result accounts for at most that, so the rest, the kernel's
+    error before rounding, stays within 2e-2 (max) and 2e-3 (mean)."""
     if w is not None and getattr(w, "q_scale", 1.0) != 1.0:
-        a = np.abs(want)
-        assert np.all(d <= OUT_MAX_ABS + a / 128.0), f"{what} max excess {np.max(d - a / 128.0):.3e}"
-        assert d.mean() <= OUT_MEAN_ABS + a.mean() / 256.0, f"{what} mean abs {d.mean():.3e}"
+        d = np.abs(got - exact)
+        hu = bf16_half_ulp(exact)
+        assert np.all(d <= OUT_MAX_ABS + hu), f"{what} max excess {np.max(d - hu):.3e}"
+        assert d.mean() <= OUT_MEAN_ABS + hu.mean(), f"{what} mean abs {d.mean():.3e} (slack {hu.mean():.2e})"
         return
+    d = np.abs(got - vo.bf16_rne(exact))
+    assert d.max() <= OUT_MAX_ABS, f"{what} max abs {d.max():.3e}"
+    assert d.mean() <= OUT_MEAN_ABS, f"{what} mean abs {d.mean():.3e}"
+
+
+def assert_gpu_outputs_close(got: np.ndarray, want: np.ndarray, what=""):
+    """Two GPU bf16 outputs of the same layer computed in different splits (the
+    spec bounds, max abs 2e-2 and mean abs 2e-3)."""
+    d = np.abs(got - want)
     assert d.max() <= OUT_MAX_ABS, f"{what} max abs {d.max():.3e}"
     assert d.mean() <= OUT_MEAN_ABS, f"{what} mean abs {d.mean():.3e}"
 

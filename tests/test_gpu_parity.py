@@ -242,7 +242,8 @@ def test_sparse_prefill_matches_oracle(case, density):
         rows = np.arange(cs, e)
         for h in range(w.hq):
             oo, ol = vo.attention_rows(cpu["q"][h, cs:e], rows, cpu["k"][h // w.group], cpu["v"][h // w.group], e,
-                                       vo.membership(e, V[h]), vo.membership(e, S[h]), w.rope_base, scale, dca)
+                                       vo.membership(e, V[h]), vo.membership(e, S[h]), w.rope_base, scale, dca,
+                                       round_out=False)
             assert_outputs_close(out[h], oo, f"{name} {density} cs={cs} h={h}", w=w)
             assert np.allclose(lse[h], ol, rtol=0, atol=2e-3), (name, density, cs, h, np.abs(lse[h] - ol).max())
         executed, useful = ctx.prefill_stats()
@@ -275,7 +276,7 @@ def test_sparse_prefill_with_large_jumps_of_the_row_max(density):
     rows = np.arange(e)
     for h in range(w.hq):
         oo, ol = vo.attention_rows(cpu["q"][h], rows, cpu["k"][0], cpu["v"][0], e, vo.membership(e, V[h]),
-                                   vo.membership(e, S[h]), w.rope_base, scale_of(w))
+                                   vo.membership(e, S[h]), w.rope_base, scale_of(w), round_out=False)
         assert_outputs_close(out[h], oo, f"jumps {density} h={h}")
         assert np.allclose(lse[h], ol, rtol=0, atol=2e-3), (density, h, np.abs(lse[h] - ol).max())
     # the spikes do move the max: most rows past a spike attend mostly to it
@@ -293,7 +294,8 @@ def test_sparse_prefill_rows_without_keys_are_zero():
     assert np.all(out[:, :5] == 0) and np.all(np.isneginf(lse[:, :5]))
     for h in range(2):
         oo, _ = vo.attention_rows(cpu["q"][h, 5:], np.arange(5, 640), cpu["k"][0], cpu["v"][0], 640,
-                                  vo.membership(640, V[h]), vo.membership(640, S[h]), w.rope_base, scale_of(w))
+                                  vo.membership(640, V[h]), vo.membership(640, S[h]), w.rope_base, scale_of(w),
+                                  round_out=False)
         assert_outputs_close(out[h, 5:], oo)
 
 
@@ -340,7 +342,8 @@ def test_layer_prefill_end_to_end(case):
                             ks_budget=w.ks_budget, tau=w.refine_tau, keep=keep)
     assert ctx.status() == vsb.VS_OK
     ref = vo.layer_prefill(cpu["q"], cpu["k"], cpu["v"], chunk=w.chunk, last_q=w.last_q, kv_budget=w.kv_budget,
-                           ks_budget=w.ks_budget, tau=w.refine_tau, base=w.rope_base, scale=scale_of(w), dca=dca)
+                           ks_budget=w.ks_budget, tau=w.refine_tau, base=w.rope_base, scale=scale_of(w), dca=dca,
+                           round_out=False)
     _check_layer(name, w, keep, ref, out)
 
 
@@ -368,7 +371,7 @@ def test_calibrated_budgets_and_fixed_budget_prefill(case):
                             tau=None, keep=keep)
     assert ctx.status() == vsb.VS_OK
     ref = vo.layer_prefill(cpu["q"], cpu["k"], cpu["v"], **{**kw, "kv_budget": kv_h, "ks_budget": ks_h, "tau": None},
-                           dca=dca)
+                           dca=dca, round_out=False)
     _check_layer(name, w, keep, ref, out)
 
 

@@ -8,7 +8,7 @@ import torch
 
 import sparse_attention_estimate_b200 as vsb
 from sparse_attention_estimate_b200 import build as vsbuild
-from tests.gpu_common import assert_outputs_close, f64
+from tests.gpu_common import assert_gpu_outputs_close, f64
 from workloads import generate_layer, small_workload
 
 pytestmark = pytest.mark.gpu
@@ -61,7 +61,7 @@ def test_streamed_from_host_matches_device_chunk_loop(name):
     got, want = f64(outs[0]), f64(ref)
     assert not np.isnan(got).any(), "rows left unwritten"
     for h in range(w.hq):
-        assert_outputs_close(got[h], want[h], f"{name} head {h}", w=w)
+        assert_gpu_outputs_close(got[h], want[h], f"{name} head {h}")
 
 
 def test_streamed_rejects_device_or_misshapen_buffers():

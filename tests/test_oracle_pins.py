@@ -105,6 +105,17 @@ def test_estimate_matches_bruteforce(rng, nr, e, d):
     assert np.allclose(a, np.array(bA), rtol=1e-12, atol=1e-15)
 
 
+def test_estimate_with_prerotated_keys_is_identical(rng):
+    q = _bf16_array(rng, (7, 128), 1.5)
+    k = _bf16_array(rng, (300, 128), 1.5)
+    kr = vo.rope(k, np.arange(300), BASE)
+    for e in (7, 123, 300):
+        a = vo.estimate(q, k, e, BASE, 0.1)
+        b = vo.estimate(q, None, e, BASE, 0.1, k_rot=kr)
+        for x, y in zip(a, b):
+            assert np.array_equal(x, y)
+
+
 def test_row_softmax_sums_to_one(rng):
     q = _bf16_array(rng, (64, 128))
     k = _bf16_array(rng, (700, 128))
@@ -150,6 +161,35 @@ def test_topk_matches_numpy_stable_argsort(rng):
     order = np.argsort(-s, kind="stable")  # stable: equal scores keep index order
     for k in [10, 333]:
         assert np.array_equal(vo.topk_sorted(s, k), np.sort(order[:k]))
+
+
+def test_kth_score_matches_stable_sort_with_ties(rng):
+    """kth_score is the score at rank k of the (score descending, index ascending)
+    order: checked against Python's stable sort on integer scores with many ties,
+    k capped at the length, and the set property around it (fewer than k scores
+    above the k-th, at least k at or above it)."""
+    s = rng.integers(0, 6, 300).astype(np.float64) / 4.0
+    order = sorted(range(300), key=lambda j: (-s[j], j))
+    for k in [1, 2, 17, 150, 299, 300, 1000]:
+        kk = min(k, 300)
+        want = s[order[kk - 1]]
+        got = vo.kth_score(s, k)
+        assert got == want, (k, got, want)
+        assert np.sum(s > got) < kk <= np.sum(s >= got)
+        assert vo.kth_score(s, k, order=vo.ranking(s)) == want
+    # a strictly increasing score: the k-th largest is the (n - k)-th element
+    inc = np.arange(50, dtype=np.float64)
+    assert vo.kth_score(inc, 5) == 45.0
+
+
+def test_select_with_precomputed_orders_is_identical(rng):
+    vert = rng.integers(0, 9, 500).astype(np.float64)
+    slash = rng.integers(0, 9, 500).astype(np.float64)
+    orders = vo.select_orders(vert, slash)
+    for kv, ks in [(1, 1), (37, 81), (500, 500), (900, 3)]:
+        a = vo.select(vert, slash, kv, ks)
+        b = vo.select(vert, slash, kv, ks, orders)
+        assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
 
 
 def test_select_matches_bruteforce_and_forces_offset0(rng):
@@ -284,6 +324,27 @@ def test_block_evaluator_equals_row_definition(rng, dca):
     o2, l2 = vo.attention_rows_dense(q[rows], rows, k, v, n, inV, inS, BASE, 0.25, dca)
     assert np.allclose(l1, l2, rtol=1e-13, atol=1e-13)
     assert np.array_equal(o1, o2) or np.max(np.abs(o1 - o2)) <= 2.0 ** -7 * np.max(np.abs(o2))
+
+
+@pytest.mark.parametrize("dca", [None, (64, 8)])
+def test_attention_rows_unrounded_and_prerotated_paths(rng, dca):
+    """round_out=False returns the float64 outputs whose bf16 rounding is the
+    default output; pre-rotated keys at the key positions change nothing."""
+    e = 150
+    q = _bf16_array(rng, (e, 16))
+    k = _bf16_array(rng, (e, 16))
+    v = _bf16_array(rng, (e, 16))
+    inV = rng.random(e) < 0.3
+    inS = rng.random(e) < 0.2
+    inS[0] = True
+    rows = np.array([0, 3, 64, 100, 149])
+    o, l = vo.attention_rows(q[rows], rows, k, v, e, inV, inS, BASE, 0.25, dca)
+    ox, lx = vo.attention_rows(q[rows], rows, k, v, e, inV, inS, BASE, 0.25, dca, round_out=False)
+    assert np.array_equal(vo.bf16_rne(ox), o) and np.array_equal(l, lx)
+    assert not np.array_equal(ox, o)  # the unrounded values carry more bits
+    kr = vo.rope(k, vo.key_positions(e, dca), BASE)
+    o2, l2 = vo.attention_rows(q[rows], rows, None, v, e, inV, inS, BASE, 0.25, dca, k_rot=kr)
+    assert np.array_equal(o2, o) and np.array_equal(l2, l)
 
 
 def test_uniform_scores_average_selected_values(rng):
@@ -488,7 +549,8 @@ ORIG_ESTIMATE = vo.estimate
 
 
 @pytest.mark.parametrize("mutant", ["rope_sign", "rope_swap", "slash_offbyone", "no_causal",
-                                    "topk_ascending", "dca_no_clip"])
+                                    "topk_ascending", "ranking_ascending", "ranking_index_descending",
+                                    "recall_forward_offsets", "dca_no_clip"])
 def test_planted_mistakes_are_caught(rng, monkeypatch, mutant):
     if mutant.startswith("rope"):
         monkeypatch.setattr(vo, "rope", _mutant_rope(mutant))
@@ -498,7 +560,19 @@ def test_planted_mistakes_are_caught(rng, monkeypatch, mutant):
         monkeypatch.setattr(vo, "estimate", _mutant_estimate_nocausal)
     elif mutant == "topk_ascending":
         monkeypatch.setattr(vo, "topk_sorted",
-                            lambda s, k: np.sort(np.lexsort((np.arange(len(s)), s))[: min(k, len(s))]))
+                            lambda s, k, order=None: np.sort(np.lexsort((np.arange(len(s)), s))[: min(k, len(s))]))
+    elif mutant == "ranking_ascending":
+        monkeypatch.setattr(vo, "ranking", lambda s: np.lexsort((np.arange(len(s)), s)))
+    elif mutant == "ranking_index_descending":
+        monkeypatch.setattr(vo, "ranking", lambda s: np.lexsort((-np.arange(len(s)), -s)))
+    elif mutant == "recall_forward_offsets":
+        def recall(a, rows, inV, inS):  # offsets read forwards: inS[j] instead of inS[i - j]
+            tot = 0.0
+            for r, i in enumerate(rows):
+                sel = inV[: i + 1] | inS[: i + 1]
+                tot += a[r, : i + 1][sel].sum()
+            return tot / len(rows)
+        monkeypatch.setattr(vo, "recall", recall)
     elif mutant == "dca_no_clip":
         monkeypatch.setattr(vo, "dca_q_position",
                             lambda i, c, C, W: [i % (C - W), i % (C - W) + C - W, C - 1][c])
@@ -512,6 +586,8 @@ def test_planted_mistakes_are_caught(rng, monkeypatch, mutant):
         lambda: test_dca_golden_table(),
         lambda: test_dca_statements_on_random_pairs(rng),
         lambda: test_layer_prefill_matches_bruteforce_chain(rng),
+        lambda: test_kth_score_matches_stable_sort_with_ties(rng),
+        lambda: test_refine_matches_bruteforce(rng, 0.6),
     ]
     caught = 0
     for p in pins:
