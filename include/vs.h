@@ -29,7 +29,9 @@
  *    positions when enabled) in its workspace and extends them as e grows. Rows
  *    [0, e) of k must not change between calls that pass the same k pointer
  *    (an append-only KV cache); call vs_context_reset() before reusing the
- *    buffer for other contents.
+ *    buffer for other contents. Every call that reuses a cached rotation
+ *    re-rotates 8 rows spread over it and compares them with the cache; a
+ *    difference is reported by vs_status_poll() as VS_ERR_DEVICE_CHECK.
  *  - Not thread-safe per context; distinct contexts are independent.
  */
 #ifndef VS_H_
@@ -155,6 +157,19 @@ VS_API vs_status vs_refine(vs_ctx* ctx, const uint16_t* q, int64_t q_rows, int64
                     float* recall, cudaStream_t stream);
 
 /*
+ * vs_calibrate_accumulate - the offline form of sparsity refinement ("Sparsity
+ * Refinement": the budgets are improved once, on a calibration sequence): after
+ * vs_refine has refined one calibration chunk from the base budgets, each head keeps
+ * the larger of its accumulated and its refined budgets,
+ *   kv_acc[h] = max(kv_acc[h], kv_budget[h]),  ks_acc[h] = max(ks_acc[h], ks_budget[h]).
+ * All four are device int32 [hq]; the caller initialises the accumulators (e.g. to 0)
+ * and passes them, once every calibration chunk is in, as the fixed budgets of
+ * vs_select for every chunk of later sequences.
+ */
+VS_API vs_status vs_calibrate_accumulate(vs_ctx* ctx, const int32_t* kv_budget, const int32_t* ks_budget,
+                                  int32_t* kv_acc, int32_t* ks_acc, cudaStream_t stream);
+
+/*
  * vs_sparse_prefill - attention of the chunk rows i in [q_pos0, e) over the
  * keys j <= i selected by the vertical-slash sets ("Sparse Attention" step 4;
  * "Algorithm": attention with DCA positions):
@@ -173,8 +188,10 @@ VS_API vs_status vs_sparse_prefill(vs_ctx* ctx, const uint16_t* q, int64_t q_row
                             uint16_t* out, float* lse_out, cudaStream_t stream);
 
 /* Counters of the last vs_sparse_prefill on this context (synchronises the
- * stream): [0] executed 128x128 (query x key) tiles summed over heads,
- * [1] selected (useful) query-key pairs summed over heads. */
+ * stream): [0] executed 128-query x 128-key tiles summed over heads (a tile is a
+ * key block, or a group of up to 128 selected vertical columns gathered from key
+ * blocks the call does not execute), [1] selected (useful) query-key pairs summed
+ * over heads. */
 VS_API vs_status vs_prefill_stats(vs_ctx* ctx, cudaStream_t stream, int64_t* out2 /* host [2] */);
 
 /* Measurement hook: when both events are non-NULL, every following
@@ -194,7 +211,8 @@ VS_API vs_status vs_set_prefill_events(vs_ctx* ctx, cudaEvent_t start, cudaEvent
  * outputs exactly as in vs_select, except that cap_v and cap_s must be >= e.
  * Scratch (thresholds and per-element levels) lives in a static device array
  * of 32 MiB per device, held by every GPU that loads the library until exit;
- * hq * 2 * round_up(e, 128) bytes plus ~hq * 512 bytes must fit, else
+ * hq * 2 * round_up(e, 128) bytes of levels plus, per head, about 2 KB and 2 KB per
+ * selection segment (at most 64 segments; 11 at 28 heads) must fit, else
  * VS_ERR_UNSUPPORTED. Nothing is allocated. The first call on a device looks up
  * the array's device address (make it before any stream capture begins); the
  * lookup is repeated when another CUDA context is current on that device, e.g.

@@ -31,7 +31,8 @@ STATUS_NAMES = {0: "VS_OK", 1: "VS_ERR_INVALID_ARG", 2: "VS_ERR_UNSUPPORTED", 3:
 EXPORTS = ("vs_workspace_size", "vs_context_create", "vs_context_destroy", "vs_context_reset",
            "vs_set_wait_limit", "dca_remap", "vs_estimate", "vs_select", "vs_refine",
            "vs_sparse_prefill", "vs_prefill_stats", "vs_status_poll", "vs_selftest_wait_timeout",
-           "vs_last_error", "vs_set_prefill_events", "vs_kernel_launches", "vs_select_noalloc")
+           "vs_last_error", "vs_set_prefill_events", "vs_kernel_launches", "vs_select_noalloc",
+           "vs_calibrate_accumulate")
 
 
 class VsError(RuntimeError):
@@ -76,6 +77,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "vs_selftest_wait_timeout": [P, U64, P],
         "vs_set_prefill_events": [P, P, P],
         "vs_select_noalloc": [I32, P, P, I64, I64, P, P, P, I32, P, P, I32, P, P],
+        "vs_calibrate_accumulate": [P, P, P, P, P, P],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -285,6 +287,11 @@ class Context:
         b = None if stop is None else ctypes.c_void_p(stop.cuda_event)
         _check(self.lib.vs_set_prefill_events(self.handle, a, b))
 
+    def calibrate_accumulate(self, kv_budget, ks_budget, kv_acc, ks_acc):
+        """kv_acc / ks_acc (int32 [hq] on the device) keep the larger budgets, in place."""
+        _check(self.lib.vs_calibrate_accumulate(self.handle, _ptr(kv_budget), _ptr(ks_budget), _ptr(kv_acc),
+                                                _ptr(ks_acc), _stream()))
+
     def selftest_wait_timeout(self, limit_ns: int):
         _check(self.lib.vs_selftest_wait_timeout(self.handle, limit_ns, _stream()))
 
@@ -306,8 +313,7 @@ def calibrate(ctx: Context, q: torch.Tensor, k: torch.Tensor, *, chunk: int, kv_
         kvb = torch.full((hq,), kv_budget, dtype=torch.int32, device=dev)
         ksb = torch.full((hq,), ks_budget, dtype=torch.int32, device=dev)
         ctx.refine(q, cs, k, e, vert, slash, lse, tau, kvb, ksb, max_iters=max_iters, full=True)
-        torch.maximum(kv_c, kvb, out=kv_c)
-        torch.maximum(ks_c, ksb, out=ks_c)
+        ctx.calibrate_accumulate(kvb, ksb, kv_c, ks_c)
     return kv_c, ks_c
 
 

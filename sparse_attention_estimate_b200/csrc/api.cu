@@ -50,6 +50,10 @@ Layout make_layout(const vs_attn_cfg& cfg, int64_t max_seq, int64_t max_chunk) {
   L.nwords = L.e_pad / 32 + kSPad + 8;
   L.npairs = L.rows_pad / (2 * kTile);
   L.nblk = L.e_pad / kTile;
+  // DCA key chunks: the gather groups never straddle one, so each has one DCA class
+  L.nkmax = cfg.dca_enabled ? ceil_div(max_seq, cfg.dca_chunk_size - cfg.dca_local_window) + 1 : 1;
+  L.gcap = L.nblk + L.nkmax + 1;
+  L.nsched = L.nblk + L.gcap;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     size_t o = off;
@@ -69,12 +73,20 @@ Layout make_layout(const vs_attn_cfg& cfg, int64_t max_seq, int64_t max_chunk) {
   L.part_s = take(static_cast<size_t>(hq) * 4 * (L.e_pad + 256) * sizeof(float));
   L.thr = take(static_cast<size_t>(hq) * 2 * kMaxLevels * 2 * sizeof(uint32_t));
   L.lvl = take(static_cast<size_t>(hq) * 2 * L.e_pad);
+  L.sel_state = take(sel_state_bytes(static_cast<int>(hq)));
+  L.sel_part = take(sel_part_bytes(static_cast<int>(hq), kRecallLevels));
   L.hist = take(static_cast<size_t>(L.nsplit_max) * hq * kMaxLevels * sizeof(float));
   L.choice = take(static_cast<size_t>(hq) * 4 * sizeof(int32_t));
   L.vbits = take(static_cast<size_t>(hq) * L.nwords * sizeof(uint32_t));
   L.sbits = take(static_cast<size_t>(hq) * L.nwords * sizeof(uint32_t));
   L.scum = take(static_cast<size_t>(hq) * (L.nwords + 1) * sizeof(uint32_t));
-  L.sched = take(static_cast<size_t>(hq) * L.npairs * L.nblk * sizeof(int32_t));
+  L.gbits = take(static_cast<size_t>(hq) * L.nwords * sizeof(uint32_t));
+  L.gcum = take(static_cast<size_t>(hq) * (L.nwords + 1) * sizeof(uint32_t));
+  L.gscan = take(static_cast<size_t>(hq) * (L.nblk + 1) * sizeof(int32_t));
+  L.glist = take(static_cast<size_t>(hq) * L.e_pad * sizeof(int32_t));
+  L.gtab = take(static_cast<size_t>(hq) * L.gcap * 4 * sizeof(int32_t));
+  L.gkoff = take(static_cast<size_t>(hq) * (L.nkmax + 1) * sizeof(int32_t));
+  L.sched = take(static_cast<size_t>(hq) * L.npairs * L.nsched * sizeof(int32_t));
   L.sched_cnt = take(static_cast<size_t>(hq) * L.npairs * sizeof(int32_t));
   L.total = off;
   return L;
@@ -117,6 +129,11 @@ using namespace vs;
 
 // ------------------------------------------------------------------ validation helpers
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static SelScratch sel_scratch(vs_ctx* c) {
+  return SelScratch{ws_ptr<uint32_t>(c, c->L.thr), ws_ptr<uint8_t>(c, c->L.lvl), c->L.e_pad,
+                    c->ws + c->L.sel_state, ws_ptr<uint32_t>(c, c->L.sel_part), c->err};
+}
 
 static vs_status check_cfg(const vs_attn_cfg* cfg) {
   VS_REQUIRE(cfg, VS_ERR_INVALID_ARG, "cfg is NULL");
@@ -328,9 +345,8 @@ extern "C" vs_status vs_select(vs_ctx* c, const float* vert, const float* slash,
   VS_REQUIRE(kv_budget && ks_budget, VS_ERR_INVALID_ARG, "budgets are NULL");
   VS_REQUIRE(e >= 1 && e <= c->max_seq && e_ld >= e, VS_ERR_INVALID_ARG, "bad e / e_ld");
   VS_TRY(check_sets(v_idx, cap_v, v_cnt, s_off, cap_s, s_cnt));
-  VS_TRY(run_thresholds(c, vert, slash, e_ld, e, kv_budget, ks_budget, 1, st));
-  VS_TRY(run_levels(c, vert, slash, e_ld, e, 1, st));
-  return run_compact(c, e, nullptr, v_idx, cap_v, v_cnt, s_off, cap_s, s_cnt, st);
+  return launch_select(sel_scratch(c), c->cfg.hq, vert, slash, e_ld, e, kv_budget, ks_budget, 1, nullptr,
+                       v_idx, cap_v, v_cnt, s_off, cap_s, s_cnt, true, true, st);
 }
 
 extern "C" vs_status vs_refine(vs_ctx* c, const uint16_t* q, int64_t q_rows, int64_t q_pos0,
@@ -356,15 +372,23 @@ extern "C" vs_status vs_refine(vs_ctx* c, const uint16_t* q, int64_t q_rows, int
   const int nlev = std::min(std::min(max_iters, kRecallLevels - 1) + 1, sat + 1);
   int nr = 0;
   VS_TRY(prepare_estimation(c, q, q_rows, q_pos0, k, k_rows, e, st, &nr));
-  VS_TRY(run_thresholds(c, vert, slash, e_ld, e, kv_budget, ks_budget, nlev, st));
-  VS_TRY(run_levels(c, vert, slash, e_ld, e, nlev, st));
+  VS_TRY(launch_select(sel_scratch(c), c->cfg.hq, vert, slash, e_ld, e, kv_budget, ks_budget, nlev, nullptr,
+                       v_idx, cap_v, v_cnt, s_off, cap_s, s_cnt, true, false, st));
   if (c->cfg.refine_dca_positions && c->dca.enabled)
     VS_TRY(run_recall_hist_dca(c, q, q_rows, q_pos0, k, k_rows, e, nr, nlev, st));
   else
     VS_TRY(run_recall_hist(c, e, nr, lse, nlev, st));
   VS_TRY(run_refine_decide(c, e, nr, nlev, tau, kv_budget, ks_budget, recall, st));
-  return run_compact(c, e, ws_ptr<int32_t>(c, c->L.choice), v_idx, cap_v, v_cnt, s_off, cap_s,
-                     s_cnt, st);
+  return launch_select(sel_scratch(c), c->cfg.hq, vert, slash, e_ld, e, kv_budget, ks_budget, nlev,
+                       ws_ptr<int32_t>(c, c->L.choice), v_idx, cap_v, v_cnt, s_off, cap_s, s_cnt, false, true,
+                       st);
+}
+
+extern "C" vs_status vs_calibrate_accumulate(vs_ctx* c, const int32_t* kv_budget, const int32_t* ks_budget,
+                                             int32_t* kv_acc, int32_t* ks_acc, cudaStream_t st) {
+  VS_TRY(check_ctx(c));
+  VS_REQUIRE(kv_budget && ks_budget && kv_acc && ks_acc, VS_ERR_INVALID_ARG, "budget pointers must not be NULL");
+  return run_budgets_max(c->cfg.hq, kv_budget, ks_budget, kv_acc, ks_acc, st);
 }
 
 extern "C" vs_status vs_sparse_prefill(vs_ctx* c, const uint16_t* q, int64_t q_rows,
@@ -421,10 +445,13 @@ extern "C" vs_status vs_status_poll(vs_ctx* c, cudaStream_t st) {
                     "error word readback"));
   VS_TRY(cuda_check(cudaStreamSynchronize(st), "status sync"));
   if (h != 0) {
-    VS_TRY(cuda_check(cudaMemsetAsync(c->err, 0, sizeof(int), st), "error word clear"));
+    VS_TRY(cuda_check(cudaMemsetAsync(c->err, 0, 3 * sizeof(int), st), "error word clear"));
     VS_TRY(cuda_check(cudaStreamSynchronize(st), "status sync"));
     if (h == kDevErrTimeout)
       return set_error(VS_ERR_TIMEOUT, "a bounded device wait ran out");
+    if (h == 5)
+      return set_error(VS_ERR_DEVICE_CHECK,
+                       "the keys changed under a cached rotation (call vs_context_reset after rewriting K)");
     return set_error(VS_ERR_DEVICE_CHECK, "device check failed (code %d)", h);
   }
   return VS_OK;

@@ -119,21 +119,163 @@ __device__ __forceinline__ uint32_t bit_prefix(const uint32_t* bits, const uint3
   return cum[w] + (r ? __popc(bits[w] & ((1u << r) - 1u)) : 0u);
 }
 
+// Selected slash offsets in [lo, hi] (inclusive, clipped to the valid offsets by the caller).
+__device__ __forceinline__ uint32_t slash_count(const uint32_t* sb, const uint32_t* sc, int64_t lo, int64_t hi) {
+  if (hi < lo) return 0u;
+  return bit_prefix(sb, sc, hi + 1 + 32 * kSPad) - bit_prefix(sb, sc, lo + 32 * kSPad);
+}
+
+// Entry of a work list: bits 0..23 key block (or gather group) index, bits 24..27 the
+// two query tiles' states (0 skip, 1 partial, 2 full), bit 28 a gather group, bit 29 a
+// key block holding gathered columns (its mask drops them) or a gather group whose
+// columns can follow some of the pair's rows (its mask is causal).
+constexpr int32_t kEntGroup = 1 << 28;
+constexpr int32_t kEntFlag = 1 << 29;
+constexpr int32_t kCntGroups = 1 << 30;  // in a list's count: the list holds gather groups
+
+// Gather plan of one head for the chunk of rows [q_pos0, e): which key blocks' vertical
+// columns are gathered into dense 128-column groups instead of executing the blocks.
+// A block's verticals cost, per pair of query tiles that can see them, either the whole
+// block (unless the block's selected offsets make the pair execute it anyway) or
+// count/128 of a gathered tile: they are gathered when that is cheaper summed over the
+// pairs. Gathered columns leave the masks of the blocks, so each selected element is
+// computed once. Writes gbits (the gathered columns' bitmap), gscan (gathered columns
+// before each block), glist (the gathered columns, ascending), and the group table:
+// consecutive runs of up to 128 gathered columns that never cross a DCA chunk boundary,
+// gkoff[k] the first group of key chunk k (gkoff[nk] the number of groups).
+__global__ void __launch_bounds__(1024) gather_plan_kernel(
+    const uint32_t* __restrict__ vbits, const uint32_t* __restrict__ sbits,
+    const uint32_t* __restrict__ scum, int64_t nwords, int64_t q_pos0, int64_t e, int npairs,
+    DcaParams dca, int64_t nblk_ws, int64_t gcap, int64_t nkmax, uint32_t* __restrict__ gbits,
+    int32_t* __restrict__ gscan, int32_t* __restrict__ glist, int4* __restrict__ gtab,
+    int32_t* __restrict__ gkoff, int64_t e_pad) {
+  const int h = blockIdx.x, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const uint32_t* vb = vbits + static_cast<int64_t>(h) * nwords;
+  const uint32_t* sb = sbits + static_cast<int64_t>(h) * nwords;
+  const uint32_t* sc = scum + static_cast<int64_t>(h) * (nwords + 1);
+  uint32_t* gb = gbits + static_cast<int64_t>(h) * nwords;
+  int32_t* gs = gscan + static_cast<int64_t>(h) * (nblk_ws + 1);
+  int32_t* gl = glist + static_cast<int64_t>(h) * e_pad;
+  int4* gt = gtab + static_cast<int64_t>(h) * gcap;
+  int32_t* gk = gkoff + static_cast<int64_t>(h) * (nkmax + 1);
+  const int64_t nb = (e + kTile - 1) / kTile;
+  // 1. decision and gathered count per block
+  for (int64_t b = tid; b < nb; b += blockDim.x) {
+    const uint4 v = *reinterpret_cast<const uint4*>(vb + 4 * b);
+    const int c = __popc(v.x) + __popc(v.y) + __popc(v.z) + __popc(v.w);
+    bool g = false;
+    if (c > 0 && c < kTile) {
+      // pairs with a row at or after the block's first key: R0 + 255 >= 128 b
+      const int64_t need = kTile * b - 255 - q_pos0;
+      const int64_t p_min = need <= 0 ? 0 : (need + 255) / 256;
+      const int64_t n_vis = npairs - p_min;
+      if (n_vis > 0) {
+        const int64_t limit = n_vis * (kTile - c);  // gather iff 128 * cover < limit
+        int64_t cover = 0;
+        for (int64_t p = p_min; p < npairs && kTile * cover < limit; ++p) {
+          const int64_t R0 = q_pos0 + 256 * p;
+          const int64_t lo = max(R0 - kTile * b - 127, static_cast<int64_t>(0));
+          const int64_t hi = min(min(R0 + 255, e - 1) - kTile * b, e - 1);
+          if (slash_count(sb, sc, lo, hi) > 0u) ++cover;
+        }
+        g = kTile * cover < limit;
+      }
+    }
+    *reinterpret_cast<uint4*>(gb + 4 * b) = g ? v : make_uint4(0u, 0u, 0u, 0u);
+    gs[b] = g ? c : 0;
+  }
+  __syncthreads();
+  // 2. exclusive scan of the counts over the blocks (gs[nb] = total)
+  __shared__ int wsum[32];
+  int running = 0;
+  for (int64_t b0 = 0; b0 < nb; b0 += blockDim.x) {
+    const int64_t b = b0 + tid;
+    const int v = b < nb ? gs[b] : 0;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) wsum[w] = x;
+    __syncthreads();
+    if (w == 0) {
+      int t = wsum[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, t, o);
+        if (lane >= o) t += y;
+      }
+      wsum[lane] = t;
+    }
+    __syncthreads();
+    if (b < nb) gs[b] = running + (w > 0 ? wsum[w - 1] : 0) + x - v;
+    running += wsum[31];
+    __syncthreads();
+  }
+  if (tid == 0) gs[nb] = running;
+  __syncthreads();
+  // 3. the gathered columns, ascending
+  for (int64_t b = tid; b < nb; b += blockDim.x) {
+    const uint4 v = *reinterpret_cast<const uint4*>(gb + 4 * b);
+    const uint32_t ws[4] = {v.x, v.y, v.z, v.w};
+    int pos = gs[b];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t m = ws[q];
+      while (m) {
+        const int x = __ffs(m) - 1;
+        m &= m - 1u;
+        gl[pos++] = static_cast<int32_t>(kTile * b + 32 * q + x);
+      }
+    }
+  }
+  // 4. groups: per DCA key chunk k (blocks [k S/128, (k+1) S/128)), runs of 128 columns
+  const int64_t sblk = dca.enabled ? dca.S / kTile : nb;  // blocks per key chunk (S % 128 == 0)
+  const int64_t nk = (nb + sblk - 1) / sblk;
+  if (tid == 0) {
+    int32_t g = 0;
+    for (int64_t k = 0; k < nk; ++k) {
+      gk[k] = g;
+      const int64_t c0 = gs[k * sblk], c1 = gs[min((k + 1) * sblk, nb)];
+      g += static_cast<int32_t>((c1 - c0 + kTile - 1) / kTile);
+    }
+    gk[nk] = g;
+  }
+  __syncthreads();
+  const int32_t ng = gk[nk];
+  for (int32_t g = tid; g < ng; g += blockDim.x) {
+    int64_t lo = 0, hi = nk - 1;  // the key chunk k with gk[k] <= g < gk[k + 1]
+    while (lo < hi) {
+      const int64_t mid = (lo + hi + 1) / 2;
+      if (gk[mid] <= g) lo = mid; else hi = mid - 1;
+    }
+    const int64_t k = lo;
+    const int64_t c0 = gs[k * sblk], c1 = gs[min((k + 1) * sblk, nb)];
+    const int64_t start = c0 + static_cast<int64_t>(g - gk[k]) * kTile;
+    const int cnt = static_cast<int>(min(static_cast<int64_t>(kTile), c1 - start));
+    gt[g] = make_int4(static_cast<int>(start), cnt, static_cast<int>(k), gl[start]);
+  }
+}
+
 // State of (query tile starting at R0, key block starting at k0): 0 skip, 1 partial, 2 full.
+// Gathered columns (gb) do not count: they are computed in their groups. *has_g tells
+// whether the block holds gathered columns (its mask must then drop them).
 __device__ __forceinline__ int tile_block_state(int64_t R0, int64_t k0, int64_t e,
                                                 const uint32_t* vb, const uint32_t* sb,
-                                                const uint32_t* sc) {
+                                                const uint32_t* sc, const uint32_t* gb,
+                                                bool* has_g) {
+  const uint4 gv = *reinterpret_cast<const uint4*>(gb + (k0 >> 5));
+  *has_g = (gv.x | gv.y | gv.z | gv.w) != 0u;
   if (R0 >= e || k0 > R0 + 127) return 0;
   const int64_t dhi_raw = R0 + 127 - k0;
   const int64_t dlo = R0 - k0 - 127 > 0 ? R0 - k0 - 127 : 0;
   const int64_t dhi = dhi_raw < e - 1 ? dhi_raw : e - 1;
-  uint32_t scount = 0;
-  if (dhi >= dlo)
-    scount = bit_prefix(sb, sc, dhi + 1 + 32 * kSPad) - bit_prefix(sb, sc, dlo + 32 * kSPad);
+  const uint32_t scount = slash_count(sb, sc, dlo, dhi);
   const bool s_all = dhi >= dlo && scount == static_cast<uint32_t>(dhi - dlo + 1);
   const uint4 v = *reinterpret_cast<const uint4*>(vb + (k0 >> 5));
-  const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
-  const bool v_all = (v.x & v.y & v.z & v.w) == 0xFFFFFFFFu;
+  const uint32_t vw[4] = {v.x & ~gv.x, v.y & ~gv.y, v.z & ~gv.z, v.w & ~gv.w};
+  const bool v_all = (vw[0] & vw[1] & vw[2] & vw[3]) == 0xFFFFFFFFu;
   const int64_t lim = dhi_raw;  // columns c <= lim can be causal for some row
   bool v_any = false;
 #pragma unroll
@@ -147,33 +289,42 @@ __device__ __forceinline__ int tile_block_state(int64_t R0, int64_t k0, int64_t 
       m = (2u << (lim - 32 * q)) - 1u;
     v_any |= (vw[q] & m) != 0u;
   }
-  if (v_all || s_all) return 2;
+  if (v_all || (s_all && !*has_g)) return 2;
   return (v_any || scount > 0) ? 1 : 0;
 }
 
+// Work list of one (pair of query tiles, head), key chunk by DCA key chunk (one chunk
+// without DCA): the gather groups of the chunk whose first column some row of the pair
+// can see, then the chunk's key blocks with a selected non-gathered element for either
+// tile. Ordered this way, the DCA class of consecutive entries changes at most twice.
 __global__ void __launch_bounds__(256) schedule_kernel(
     const uint32_t* __restrict__ vbits, const uint32_t* __restrict__ sbits,
-    const uint32_t* __restrict__ scum, int64_t nwords, int64_t q_pos0, int64_t e, int npairs_ws,
-    int64_t nblk_ws, int32_t* __restrict__ sched, int32_t* __restrict__ sched_cnt,
-    unsigned long long* stats) {
+    const uint32_t* __restrict__ scum, const uint32_t* __restrict__ gbits,
+    const int4* __restrict__ gtab, const int32_t* __restrict__ gkoff,
+    const int32_t* __restrict__ glist, int64_t e_pad, int64_t nwords, int64_t q_pos0, int64_t e,
+    DcaParams dca, int64_t gcap, int64_t nkmax, int npairs_ws, int64_t nsched,
+    int32_t* __restrict__ sched, int32_t* __restrict__ sched_cnt, unsigned long long* stats) {
   const int pair = blockIdx.x, h = blockIdx.y, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const uint32_t* vb = vbits + static_cast<int64_t>(h) * nwords;
   const uint32_t* sb = sbits + static_cast<int64_t>(h) * nwords;
   const uint32_t* sc = scum + static_cast<int64_t>(h) * (nwords + 1);
+  const uint32_t* gb = gbits + static_cast<int64_t>(h) * nwords;
+  const int4* gt = gtab + static_cast<int64_t>(h) * gcap;
+  const int32_t* gk = gkoff + static_cast<int64_t>(h) * (nkmax + 1);
   const int64_t R0 = q_pos0 + static_cast<int64_t>(pair) * 256;
   const int64_t last_row = (e - 1 < R0 + 255) ? e - 1 : R0 + 255;
   const int64_t nb = last_row / kTile + 1;
-  int32_t* out = sched + (static_cast<int64_t>(h) * npairs_ws + pair) * nblk_ws;
+  const int64_t sblk = dca.enabled ? dca.S / kTile : nb;
+  const int64_t nk = (nb + sblk - 1) / sblk;
+  const int64_t nk_all = ((e + kTile - 1) / kTile + sblk - 1) / sblk;  // key chunks of the plan
+  int32_t* out = sched + (static_cast<int64_t>(h) * npairs_ws + pair) * nsched;
+  auto gl_last = [&](int hh, const int4& d) {  // last column of a group
+    return static_cast<int64_t>(glist[static_cast<int64_t>(hh) * e_pad + d.x + d.y - 1]);
+  };
   __shared__ int wsum[8];
-  int running = 0;
-  for (int64_t b0 = 0; b0 < nb; b0 += 256) {
-    const int64_t b = b0 + tid;
-    int flags = 0;
-    if (b < nb) {
-      const int64_t k0 = b * kTile;
-      flags = tile_block_state(R0, k0, e, vb, sb, sc) | (tile_block_state(R0 + 128, k0, e, vb, sb, sc) << 2);
-    }
-    const int f = flags != 0;
+  int running = 0, groups = 0;
+  // block-wide compaction of one batch of 256 candidate entries (flagged when non-zero)
+  auto emit = [&](bool f, int32_t entry) {
     const uint32_t bal = __ballot_sync(0xffffffffu, f);
     if (lane == 0) wsum[w] = __popc(bal);
     __syncthreads();
@@ -181,12 +332,53 @@ __global__ void __launch_bounds__(256) schedule_kernel(
     for (int i = 0; i < w; ++i) base += wsum[i];
     int total = 0;
     for (int i = 0; i < 8; ++i) total += wsum[i];
-    if (f) out[base + __popc(bal & ((1u << lane) - 1u))] = static_cast<int32_t>(b) | (flags << 24);
+    if (f) out[base + __popc(bal & ((1u << lane) - 1u))] = entry;
     running += total;
     __syncthreads();
+  };
+  for (int64_t k = 0; k < nk; ++k) {
+    // gather groups of key chunk k
+    const int32_t g0 = k < nk_all ? gk[k] : 0, g1 = k < nk_all ? gk[k + 1] : 0;
+    for (int32_t gb0 = g0; gb0 < g1; gb0 += 256) {
+      const int32_t g = gb0 + tid;
+      bool f = false;
+      int32_t entry = 0;
+      const int before = running;
+      if (g < g1) {
+        const int4 d = gt[g];  // start, count, key chunk, first column
+        const int64_t first_col = d.w;
+        const int64_t last_col = gl_last(h, d);
+        f = first_col <= last_row;
+        int flags = 0;
+        for (int t = 0; t < 2; ++t) {
+          const int64_t r0 = R0 + t * kTile;
+          if (r0 >= e || first_col > min(r0 + 127, e - 1)) continue;  // no row of the tile sees it
+          // full: 128 columns, all before the tile's first row
+          flags |= (d.y == kTile && last_col < r0 ? 2 : 1) << (2 * t);
+        }
+        // causal mask needed when a column of the group can follow one of the pair's rows
+        entry = g | kEntGroup | (flags << 24) | (last_col >= R0 ? kEntFlag : 0);
+      }
+      emit(f, entry);
+      groups += running - before;
+    }
+    // key blocks of key chunk k
+    const int64_t b_lo = k * sblk, b_hi = min((k + 1) * sblk, nb);
+    for (int64_t b0 = b_lo; b0 < b_hi; b0 += 256) {
+      const int64_t b = b0 + tid;
+      int flags = 0;
+      bool hg0 = false, hg1 = false;
+      if (b < b_hi) {
+        const int64_t k0 = b * kTile;
+        flags = tile_block_state(R0, k0, e, vb, sb, sc, gb, &hg0) |
+                (tile_block_state(R0 + 128, k0, e, vb, sb, sc, gb, &hg1) << 2);
+      }
+      emit(flags != 0, static_cast<int32_t>(b) | (flags << 24) | (hg0 ? kEntFlag : 0));
+    }
   }
   if (tid == 0) {
-    sched_cnt[static_cast<int64_t>(h) * npairs_ws + pair] = running;
+    // the list's length, and bit 30 when it holds gather groups
+    sched_cnt[static_cast<int64_t>(h) * npairs_ws + pair] = running | (groups > 0 ? kCntGroups : 0);
     atomicAdd(stats, 2ull * static_cast<unsigned long long>(running));
   }
 }
@@ -200,10 +392,23 @@ struct AttnParams {
   const int32_t* sched;
   const int32_t* sched_cnt;
   int npairs_ws;
-  int64_t nblk_ws;
+  int64_t nsched;
   const uint32_t* vbits;
   const uint32_t* sbits;
   int64_t nwords;
+  // gathered vertical columns: bitmap and prefix counts [hq][nwords], the columns
+  // [hq][e_pad] and the groups [hq][gcap] (start, count, DCA key chunk, first column)
+  const uint32_t* gbits;
+  const uint32_t* gcum;
+  const int32_t* glist;
+  const int4* gtab;
+  int64_t e_pad, gcap;
+  int dca_sblk;  // key blocks per DCA chunk (S / 128), 0 without DCA
+  // row sources of the gathered groups: rotated keys and values, [hkv][rows][128]
+  const uint16_t* k_rot;
+  int64_t k_rows;
+  const uint16_t* v;
+  int64_t v_rows;
   uint16_t* out;
   int64_t out_rows;
   float* lse_out;
@@ -220,6 +425,7 @@ struct __align__(1024) AttnSmem {
   uint64_t s_full[2], p_full[2], o_final, drain;
   uint32_t tmem_base;
   int abort_word;
+  int gather_ok;  // a stage wait's outcome, shared among the gather threads
 };
 
 __device__ __forceinline__ float ex2a(float x) {
@@ -234,12 +440,20 @@ __device__ __forceinline__ void drain_wait_a(uint64_t* bar, uint32_t parity, uin
     if (globaltimer_ns() - t0 > limit) break;
 }
 
-// DCA class of (query tile starting at R0, key block starting at k0): 0 intra,
-// 1 successive, 2 inter (always 0 without DCA).
-__device__ __forceinline__ int dca_class(int64_t R0, int64_t k0, const DcaParams& d) {
-  if (!d.enabled) return 0;
-  const int64_t bi = R0 / d.S, bj = k0 / d.S;
-  return bi == bj ? 0 : (bi == bj + 1 ? 1 : 2);
+// DCA class of (query tile in DCA chunk qc, keys of DCA chunk kc): 0 intra,
+// 1 successive, 2 inter (always 0 without DCA, where every chunk index is 0).
+__device__ __forceinline__ int dca_class(int qc, int kc) {
+  return qc == kc ? 0 : (qc == kc + 1 ? 1 : 2);
+}
+
+// DCA chunk of a work-list entry's keys: a key block's (the chunk stride is sblk
+// blocks), or a gather group's (groups never straddle a chunk). 32-bit arithmetic:
+// the issuing threads run this for every entry.
+__device__ __forceinline__ int entry_kchunk(int32_t ent, const int4* gtab, int64_t gcap, int h, int sblk) {
+  if (sblk == 0) return 0;  // no DCA
+  const uint32_t idx = static_cast<uint32_t>(ent) & 0xFFFFFFu;
+  if (ent & kEntGroup) return gtab[static_cast<int64_t>(h) * gcap + idx].z;
+  return static_cast<int>(idx / static_cast<uint32_t>(sblk));
 }
 
 __global__ void __launch_bounds__(kAttnThreads, 1)
@@ -260,8 +474,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int pair = p.npairs - 1 - rg / p.g;
   const int h = hk * p.g + rg % p.g;
   const int64_t R0 = p.q_pos0 + static_cast<int64_t>(pair) * 256;  // tile 0's first row
-  const int32_t* list = p.sched + (static_cast<int64_t>(h) * p.npairs_ws + pair) * p.nblk_ws;
-  const int n = p.sched_cnt[static_cast<int64_t>(h) * p.npairs_ws + pair];
+  const int32_t* list = p.sched + (static_cast<int64_t>(h) * p.npairs_ws + pair) * p.nsched;
+  // DCA chunks of the two query tiles (fixed for the CTA)
+  const int qc0 = p.dca.enabled ? static_cast<int>(R0 / p.dca.S) : 0;
+  const int qc1 = p.dca.enabled ? static_cast<int>((R0 + kTile) / p.dca.S) : 0;
+  const int cnt_raw = p.sched_cnt[static_cast<int64_t>(h) * p.npairs_ws + pair];
+  const int n = cnt_raw & (kCntGroups - 1);
+  const bool has_groups = (cnt_raw & kCntGroups) != 0;
   volatile int* abort_word = &s.abort_word;
 
   if (tid == 0) {
@@ -300,34 +519,45 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tma_prefetch_desc(&tmV);
         int cls[2];
         int qchg[2] = {0, 0};
-        const int64_t kb0 = static_cast<int64_t>(list[0] & 0xFFFFFF) * kTile;
+        const int kc0 = entry_kchunk(list[0], p.gtab, p.gcap, h, p.dca_sblk);
         for (int t = 0; t < 2; ++t) {
-          cls[t] = dca_class(R0 + t * kTile, kb0, p.dca);
+          cls[t] = dca_class(t ? qc1 : qc0, kc0);
           mbar_arrive_expect_tx(&s.q_full[t], 2 * kTileBytes);
           const int qrow = pair * 256 + t * kTile;
           const int qh = cls[t] * p.hq + h;
           tma_load_3d(s.q[t][0], &tmQ, &s.q_full[t], 0, qrow, qh);
           tma_load_3d(s.q[t][1], &tmQ, &s.q_full[t], 64, qrow, qh);
         }
-        int kiss[2] = {0, 0}, viss[2] = {0, 0};
+        // per stage: entries seen so far (TMA or gather, each completes one phase of the
+        // stage's full barriers) and the phase of the last TMA load issued (-1: none), for
+        // draining the copies in flight when the CTA aborts
+        int nst[2] = {0, 0}, kph[2] = {-1, -1}, vph[2] = {-1, -1};
         bool ok = true;
         int32_t ent = list[0];  // schedule entries are read one block ahead of use
         for (int j = 0; j < n && ok; ++j) {
-          const int b = ent & 0xFFFFFF;
+          const int32_t cur = ent;
+          const int b = cur & 0xFFFFFF;
+          const bool grp = (cur & kEntGroup) != 0;  // a gather group: warps 2-3 load its K and V
           ent = j + 1 < n ? ld_keep_s32(list + j + 1) : 0;
           const int st = j & 1;
-          // K(j) first: the MMA warp releases a Q tile only after issuing S0(j)
-          if (j >= 2) ok = mbar_wait(&s.k_empty[st], ((j >> 1) - 1) & 1, abort_word, p.dc.err);
+          // K(j) first: the MMA warp releases a Q tile only after issuing S0(j).
+          // Both loaders (this one and the gather warps) wait for every entry's stage to
+          // empty, their own entries or not: a parity wait is exact only for the phase
+          // right after the last one waited for.
+          if (j >= 2) ok = mbar_wait(&s.k_empty[st], ((j >> 1) - 1) & 1, abort_word, p.dc.err, 1, j);
           if (!ok) break;
-          mbar_arrive_expect_tx(&s.k_full[st], 2 * kTileBytes);
-          tma_load_3d(s.k[st][0], &tmK, &s.k_full[st], 0, b * kTile, hk);
-          tma_load_3d(s.k[st][1], &tmK, &s.k_full[st], 64, b * kTile, hk);
-          ++kiss[st];
+          if (!grp) {
+            mbar_arrive_expect_tx(&s.k_full[st], 2 * kTileBytes);
+            tma_load_3d(s.k[st][0], &tmK, &s.k_full[st], 0, b * kTile, hk);
+            tma_load_3d(s.k[st][1], &tmK, &s.k_full[st], 64, b * kTile, hk);
+            kph[st] = nst[st];
+          }
           if (j > 0) {
+            const int kc = entry_kchunk(cur, p.gtab, p.gcap, h, p.dca_sblk);
             for (int t = 0; t < 2 && ok; ++t) {
-              const int c = dca_class(R0 + t * kTile, static_cast<int64_t>(b) * kTile, p.dca);
+              const int c = dca_class(t ? qc1 : qc0, kc);
               if (c != cls[t]) {
-                ok = mbar_wait(&s.q_empty[t], qchg[t] & 1, abort_word, p.dc.err);
+                ok = mbar_wait(&s.q_empty[t], qchg[t] & 1, abort_word, p.dc.err, 2 + t, j);
                 if (!ok) break;
                 ++qchg[t];
                 cls[t] = c;
@@ -339,18 +569,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
             if (!ok) break;
           }
-          if (j >= 2) ok = mbar_wait(&s.v_empty[st], ((j >> 1) - 1) & 1, abort_word, p.dc.err);
-          if (!ok) break;
+          if (j >= 2) ok = mbar_wait(&s.v_empty[st], ((j >> 1) - 1) & 1, abort_word, p.dc.err, 4, j);
+          if (!ok || grp) {
+            ++nst[st];
+            if (!ok) break;
+            continue;
+          }
           mbar_arrive_expect_tx(&s.v_full[st], 2 * kTileBytes);
           tma_load_3d(s.v[st][0], &tmV, &s.v_full[st], 0, b * kTile, hk);
           tma_load_3d(s.v[st][1], &tmV, &s.v_full[st], 64, b * kTile, hk);
-          ++viss[st];
+          vph[st] = nst[st];
+          ++nst[st];
         }
         if (!ok) {  // let every issued copy land before the CTA exits
+          // A stage's TMA load is issued only after every earlier phase of its barrier has
+          // completed, so the phase of the last one is the barrier's current phase.
           for (int t = 0; t < 2; ++t) drain_wait_a(&s.q_full[t], qchg[t] & 1, p.dc.wait_ns);
           for (int st = 0; st < 2; ++st) {
-            if (kiss[st] > 0) drain_wait_a(&s.k_full[st], (kiss[st] - 1) & 1, p.dc.wait_ns);
-            if (viss[st] > 0) drain_wait_a(&s.v_full[st], (viss[st] - 1) & 1, p.dc.wait_ns);
+            if (kph[st] >= 0) drain_wait_a(&s.k_full[st], kph[st] & 1, p.dc.wait_ns);
+            if (vph[st] >= 0) drain_wait_a(&s.v_full[st], vph[st] & 1, p.dc.wait_ns);
           }
         }
       }
@@ -363,9 +600,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const uint32_t tS[2] = {tbase, tbase + 128};
           const uint32_t tO[2] = {tbase + 256, tbase + 384};
           int cls[2], qph[2] = {1, 1};
-          const int64_t kb0 = static_cast<int64_t>(list[0] & 0xFFFFFF) * kTile;
-          cls[0] = dca_class(R0, kb0, p.dca);
-          cls[1] = dca_class(R0 + kTile, kb0, p.dca);
+          const int kc0 = entry_kchunk(list[0], p.gtab, p.gcap, h, p.dca_sblk);
+          cls[0] = dca_class(qc0, kc0);
+          cls[1] = dca_class(qc1, kc0);
           int32_t ent1 = n > 1 ? list[1] : 0;  // entry of block j + 1, read a block ahead
           // descriptor words of the operand tiles (K-major Q and K, MN-major V; 128-byte swizzle)
           const uint32_t dhi = smem_desc_sw128_hi(1024);
@@ -389,9 +626,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             for (int kk = 0; kk < 8; ++kk)  // K-step of 16 keys: 8 TMEM columns of P, 2048 bytes of V
               mma_bf16_ts_w(tO[t], tS[t] + kk * 8, b + kk * (2048 >> 4), dhi, id_pv, (acc || kk > 0) ? 1u : 0u);
           };
-          bool ok = mbar_wait(&s.q_full[0], 0, abort_word, p.dc.err) &&
-                    mbar_wait(&s.q_full[1], 0, abort_word, p.dc.err) &&
-                    mbar_wait(&s.k_full[0], 0, abort_word, p.dc.err);
+          bool ok = mbar_wait(&s.q_full[0], 0, abort_word, p.dc.err, 16, 0) &&
+                    mbar_wait(&s.q_full[1], 0, abort_word, p.dc.err, 17, 0) &&
+                    mbar_wait(&s.k_full[0], 0, abort_word, p.dc.err, 18, 0);
           if (ok) {
             tc_fence_after_sync();
             issue_qk(0, 0);
@@ -404,24 +641,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const int st = j & 1;
             const bool more = j + 1 < n;
             const int st1 = (j + 1) & 1;
-            const int64_t kb1 = more ? static_cast<int64_t>(ent1 & 0xFFFFFF) * kTile : 0;
+            const int kc1 = more ? entry_kchunk(ent1, p.gtab, p.gcap, h, p.dca_sblk) : 0;
             ent1 = j + 2 < n ? ld_keep_s32(list + j + 2) : 0;
-            const int c0 = more ? dca_class(R0, kb1, p.dca) : cls[0];
-            const int c1 = more ? dca_class(R0 + kTile, kb1, p.dca) : cls[1];
+            const int c0 = more ? dca_class(qc0, kc1) : cls[0];
+            const int c1 = more ? dca_class(qc1, kc1) : cls[1];
             // V(j) and K(j+1) normally landed long ago: wait for them before P_0(j), so
             // that PV_t(j) and S_t(j + 1) go to the tensor pipe back to back once P_t(j)
             // is stored (the pipe runs dry while this thread does anything else)
-            ok = mbar_wait(&s.v_full[st], (j >> 1) & 1, abort_word, p.dc.err) &&
-                 (!more || mbar_wait(&s.k_full[st1], ((j + 1) >> 1) & 1, abort_word, p.dc.err));
+            ok = mbar_wait(&s.v_full[st], (j >> 1) & 1, abort_word, p.dc.err, 5, j) &&
+                 (!more || mbar_wait(&s.k_full[st1], ((j + 1) >> 1) & 1, abort_word, p.dc.err, 6, j));
             // tile 0
-            ok = ok && mbar_wait(&s.p_full[0], j & 1, abort_word, p.dc.err);
+            ok = ok && mbar_wait(&s.p_full[0], j & 1, abort_word, p.dc.err, 7, j);
             if (!ok) break;
             tc_fence_after_sync();
             issue_pv(0, st, j > 0);
             if (more) {
               if (c0 != cls[0]) {  // the tile's DCA class changes: wait for Q_0 at the new rotation
                 mma_commit(&s.q_empty[0]);
-                ok = mbar_wait(&s.q_full[0], qph[0] & 1, abort_word, p.dc.err);
+                ok = mbar_wait(&s.q_full[0], qph[0] & 1, abort_word, p.dc.err, 8, j);
                 ++qph[0];
                 cls[0] = c0;
                 if (!ok) break;
@@ -431,7 +668,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               mma_commit(&s.s_full[0]);
             }
             // tile 1
-            ok = mbar_wait(&s.p_full[1], j & 1, abort_word, p.dc.err);
+            ok = mbar_wait(&s.p_full[1], j & 1, abort_word, p.dc.err, 9, j);
             if (!ok) break;
             tc_fence_after_sync();
             issue_pv(1, st, j > 0);
@@ -439,7 +676,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             if (more) {
               if (c1 != cls[1]) {
                 mma_commit(&s.q_empty[1]);
-                ok = mbar_wait(&s.q_full[1], qph[1] & 1, abort_word, p.dc.err);
+                ok = mbar_wait(&s.q_full[1], qph[1] & 1, abort_word, p.dc.err, 10, j);
                 ++qph[1];
                 cls[1] = c1;
                 if (!ok) break;
@@ -454,6 +691,62 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           drain_wait_a(&s.drain, 0, p.dc.wait_ns);
         }
         mbar_arrive(&s.o_final);
+      }
+    } else {
+      // ------------------------------------------------------------ gather loader (warps 2-3)
+      // For each gather group of the list: the 128 gathered columns' rotated K rows and
+      // V rows, copied 16 bytes at a time into the stage's tiles in the 128-byte-swizzled
+      // layout the TMA loads produce (rows past the group's count repeat its first
+      // column; their scores are masked). Thread g copies tile rows g and g + 64.
+      const int gtid = tid - 64;
+      const int32_t* gl = p.glist + static_cast<int64_t>(h) * p.e_pad;
+      int32_t ent = n > 0 ? list[0] : 0;
+      bool ok = has_groups;  // lists without groups are the TMA producer's alone
+      // Every entry's stage-empty phases are waited for (by thread 0, the outcome shared
+      // through the named barrier), as in the TMA producer: a parity wait is exact only
+      // for the phase right after the last one waited for.
+      for (int j = 0; j < n && ok; ++j) {
+        const int32_t cur = ent;
+        ent = j + 1 < n ? ld_keep_s32(list + j + 1) : 0;
+        const bool grp = (cur & kEntGroup) != 0;
+        const int st = j & 1;
+        int64_t col[2] = {0, 0};
+        if (grp) {
+          const int4 d = p.gtab[static_cast<int64_t>(h) * p.gcap + (cur & 0xFFFFFF)];  // start, count, key chunk, first column
+          col[0] = gl[d.x + (gtid < d.y ? gtid : 0)];
+          col[1] = gl[d.x + (gtid + 64 < d.y ? gtid + 64 : 0)];
+        }
+        for (int kvh = 0; kvh < 2 && ok; ++kvh) {  // K rows into k[st], then V rows into v[st]
+          if (j >= 2) {
+            if (gtid == 0)
+              s.gather_ok = mbar_wait(kvh == 0 ? &s.k_empty[st] : &s.v_empty[st], ((j >> 1) - 1) & 1, abort_word,
+                                      p.dc.err, 11 + kvh, j)
+                                ? 1
+                                : 0;
+            named_barrier_sync(1, 64);
+            ok = s.gather_ok != 0;
+            named_barrier_sync(1, 64);  // every thread has read the outcome before the next wait
+          }
+          if (!ok) break;  // uniform over the 64 threads: nothing was copied
+          if (!grp) continue;
+          const uint16_t* base = kvh == 0 ? p.k_rot : p.v;
+          const int64_t rows = kvh == 0 ? p.k_rows : p.v_rows;
+          bf16 (*dst)[kTile * 64] = kvh == 0 ? s.k[st] : s.v[st];
+#pragma unroll
+          for (int rr = 0; rr < 2; ++rr) {
+            const int r = gtid + 64 * rr;
+            const uint16_t* src = base + (static_cast<int64_t>(hk) * rows + col[rr]) * kD;
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              char* d8 = reinterpret_cast<char*>(&dst[c >> 3][0]) + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+              cp_async_16(d8, src + c * 8);
+            }
+          }
+          cp_async_wait_all();
+          fence_proxy_async_smem();  // the MMA reads these tiles through the async proxy
+          named_barrier_sync(1, 64);
+          if (gtid == 0) mbar_arrive(kvh == 0 ? &s.k_full[st] : &s.v_full[st]);
+        }
       }
     }
   } else {
@@ -476,10 +769,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       ent = j + 1 < n ? ld_keep_s32(list + j + 1) : 0;
       const int64_t k0 = static_cast<int64_t>(entry & 0xFFFFFF) * kTile;
       const int state = (entry >> (24 + 2 * t)) & 3;
-      // element mask of this row over the block's 128 keys
+      // element mask of this row over the block's (or gather group's) 128 keys
       uint32_t mw[4];
       if (state == 0 || i >= p.e) {
         mw[0] = mw[1] = mw[2] = mw[3] = 0u;
+      } else if (entry & kEntGroup) {
+        // gather group: its first `count` columns, those at or before this row when the
+        // group reaches into the pair's rows (columns ascending: a prefix of the group)
+        const int4 d = p.gtab[static_cast<int64_t>(h) * p.gcap + (entry & 0xFFFFFF)];
+        int nvalid = d.y;
+        if (entry & kEntFlag) {
+          const int64_t wi = static_cast<int64_t>(h) * p.nwords + (i >> 5);
+          const int64_t upto = static_cast<int64_t>(p.gcum[wi + h]) +  // gcum rows hold nwords + 1 entries
+                               __popc(p.gbits[wi] & ((2u << static_cast<int>(i & 31)) - 1u));  // gathered columns <= i
+          const int64_t nv = upto - d.x;
+          nvalid = nv < 0 ? 0 : (nv > d.y ? d.y : static_cast<int>(nv));
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          mw[q] = nvalid >= 32 * (q + 1) ? 0xFFFFFFFFu : (nvalid > 32 * q ? (1u << (nvalid - 32 * q)) - 1u : 0u);
       } else {
         if (state == 2) {
           mw[0] = mw[1] = mw[2] = mw[3] = 0xFFFFFFFFu;
@@ -498,6 +806,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           mw[1] = vv.y | __brev(x[2]);
           mw[2] = vv.z | __brev(x[1]);
           mw[3] = vv.w | __brev(x[0]);
+          if (entry & kEntFlag) {  // gathered columns are computed in their groups
+            const uint4 gv = *reinterpret_cast<const uint4*>(p.gbits + static_cast<int64_t>(h) * p.nwords + (k0 >> 5));
+            mw[0] &= ~gv.x;
+            mw[1] &= ~gv.y;
+            mw[2] &= ~gv.z;
+            mw[3] &= ~gv.w;
+          }
         }
         const int64_t lim = i - k0;  // causal: column c <= i - k0
         if (lim < 127) {
@@ -514,7 +829,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
         }
       }
-      ok = __all_sync(0xffffffffu, mbar_wait(&s.s_full[t], j & 1, abort_word, p.dc.err));
+      ok = __all_sync(0xffffffffu, mbar_wait(&s.s_full[t], j & 1, abort_word, p.dc.err, 13 + t, j));
       if (!ok) break;
       tc_fence_after_sync();
       useful += __popc(mw[0]) + __popc(mw[1]) + __popc(mw[2]) + __popc(mw[3]);
@@ -616,7 +931,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (lane == 0) mbar_arrive(&s.p_full[t]);
     }
     // ---------------------------------------------------------- epilogue
-    const bool fin = __all_sync(0xffffffffu, mbar_wait(&s.o_final, 0, abort_word, p.dc.err));
+    const bool fin = __all_sync(0xffffffffu, mbar_wait(&s.o_final, 0, abort_word, p.dc.err, 15, 0));
     tc_fence_after_sync();
     if (fin && ok) {
       const float inv = l_run > 0.f ? 1.0f / l_run : 0.f;
@@ -694,10 +1009,25 @@ vs_status run_sparse_prefill(vs_ctx* c, const uint16_t* q, int64_t q_rows, int64
   s = launched("prefix_popc_kernel launch");
   if (s != VS_OK) return s;
   const int npairs = static_cast<int>(ceil_div(nrows, 256));
-  schedule_kernel<<<dim3(npairs, hq), 256, 0, st>>>(vbits, sbits, scum, L.nwords, q_pos0, e,
-                                                   static_cast<int>(L.npairs), L.nblk,
-                                                   ws_ptr<int32_t>(c, L.sched),
-                                                   ws_ptr<int32_t>(c, L.sched_cnt), c->stats);
+  // vertical columns gathered into dense groups where that beats executing their blocks
+  uint32_t* gbits = ws_ptr<uint32_t>(c, L.gbits);
+  uint32_t* gcum = ws_ptr<uint32_t>(c, L.gcum);
+  s = cuda_check(cudaMemsetAsync(gbits, 0, static_cast<size_t>(hq) * L.nwords * 4, st), "gather bitmap clear");
+  if (s != VS_OK) return s;
+  gather_plan_kernel<<<hq, 1024, 0, st>>>(vbits, sbits, scum, L.nwords, q_pos0, e, npairs, c->dca, L.nblk,
+                                          L.gcap, L.nkmax, gbits, ws_ptr<int32_t>(c, L.gscan),
+                                          ws_ptr<int32_t>(c, L.glist), ws_ptr<int4>(c, L.gtab),
+                                          ws_ptr<int32_t>(c, L.gkoff), L.e_pad);
+  s = launched("gather_plan_kernel launch");
+  if (s != VS_OK) return s;
+  prefix_popc_kernel<<<hq, 1024, 0, st>>>(gbits, L.nwords, gcum);
+  s = launched("prefix_popc_kernel launch");
+  if (s != VS_OK) return s;
+  schedule_kernel<<<dim3(npairs, hq), 256, 0, st>>>(
+      vbits, sbits, scum, gbits, ws_ptr<int4>(c, L.gtab), ws_ptr<int32_t>(c, L.gkoff),
+      ws_ptr<int32_t>(c, L.glist), L.e_pad, L.nwords, q_pos0, e, c->dca, L.gcap, L.nkmax,
+      static_cast<int>(L.npairs), L.nsched, ws_ptr<int32_t>(c, L.sched), ws_ptr<int32_t>(c, L.sched_cnt),
+      c->stats);
   s = launched("schedule launch");
   if (s != VS_OK) return s;
   // tensor maps
@@ -718,10 +1048,21 @@ vs_status run_sparse_prefill(vs_ctx* c, const uint16_t* q, int64_t q_rows, int64
   ap.sched = ws_ptr<int32_t>(c, L.sched);
   ap.sched_cnt = ws_ptr<int32_t>(c, L.sched_cnt);
   ap.npairs_ws = static_cast<int>(L.npairs);
-  ap.nblk_ws = L.nblk;
+  ap.nsched = L.nsched;
   ap.vbits = vbits;
   ap.sbits = sbits;
   ap.nwords = L.nwords;
+  ap.gbits = gbits;
+  ap.gcum = gcum;
+  ap.glist = ws_ptr<int32_t>(c, L.glist);
+  ap.gtab = ws_ptr<int4>(c, L.gtab);
+  ap.e_pad = L.e_pad;
+  ap.gcap = L.gcap;
+  ap.dca_sblk = dca ? static_cast<int>(c->dca.S / kTile) : 0;
+  ap.k_rot = reinterpret_cast<const uint16_t*>(c->ws + (dca ? L.k_dca : L.k_cont));
+  ap.k_rows = c->max_seq;
+  ap.v = v;
+  ap.v_rows = kv_rows;
   ap.out = out;
   ap.out_rows = q_rows;
   ap.lse_out = lse_out;

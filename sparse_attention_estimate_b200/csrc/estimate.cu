@@ -357,7 +357,21 @@ __global__ void __launch_bounds__(kEstThreads, 1)
                   uint32_t aw[8];
 #pragma unroll
                   for (int q = 0; q < 8; ++q) aw[q] = __funnelshift_r(wv[q], wv[q + 1], sh);
-                  bin_elements([&](int x) { return (aw[(31 - x) >> 2] >> (8 * ((31 - x) & 3))) & 0xFFu; });
+                  if (nlev < static_cast<uint32_t>(kBinLevels)) {
+                    // Four elements per byte-SIMD step: columns 4q..4q+3 have their vertical
+                    // levels in vw[q] and their offsets' levels, byte-reversed, in aw[7 - q];
+                    // an element's level is the smaller one, and levels at or past nlev (never
+                    // selected) all go to bin nlev, which no level reads: no branch per element.
+                    const uint32_t cap4 = nlev * 0x01010101u;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                      const uint32_t l4 = __vminu4(__vminu4(vw[q], __byte_perm(aw[7 - q], 0u, 0x0123)), cap4);
+#pragma unroll
+                      for (int b = 0; b < 4; ++b) bins[((l4 >> (8 * b)) & 0xFFu) * kTile] += v[4 * q + b];
+                    }
+                  } else {
+                    bin_elements([&](int x) { return (aw[(31 - x) >> 2] >> (8 * ((31 - x) & 3))) & 0xFFu; });
+                  }
                 } else {
                   bin_elements([&](int x) {
                     const int64_t d = irow - (j0 + x);

@@ -58,15 +58,24 @@ struct Layout {
   size_t part_s;              // slash partial sums [hq][2 halves][2 lo/hi][e_pad + 128]
   size_t thr;                 // selection thresholds [hq][2][kMaxLevels] (key, take)
   size_t lvl;                 // levels [hq][2][max_seq] uint8
+  size_t sel_state, sel_part; // radix-select state and per-segment histograms
   size_t hist;                // recall histograms [nsplit_max][hq][kMaxLevels]
   size_t choice;              // chosen level per head [hq] + flags
   size_t vbits, sbits, scum;  // bitmaps [hq][nwords] and slash prefix counts
-  size_t sched, sched_cnt;    // block lists [hq][npairs][nblk] and counts [hq][npairs]
+  size_t gbits, gcum;         // gathered vertical columns [hq][nwords] and their prefix counts
+  size_t gscan;               // gathered columns before each key block [hq][nblk + 1]
+  size_t glist;               // gathered columns, ascending [hq][e_pad]
+  size_t gtab;                // gather groups [hq][gcap] (start, count, DCA key chunk, first column)
+  size_t gkoff;               // first group of each DCA key chunk [hq][nkmax + 1]
+  size_t sched, sched_cnt;    // work lists [hq][npairs][nsched] and counts [hq][npairs]
   size_t total;
   int64_t rows_pad;           // max_chunk rounded up to 256
   int64_t e_pad;              // max_seq rounded up to 128
   int64_t nwords;             // bitmap words per head (incl. padding)
   int64_t npairs, nblk;       // query-tile pairs per chunk, key blocks per sequence
+  int64_t nkmax;              // DCA key chunks a sequence can span (1 without DCA)
+  int64_t gcap;               // gather groups per head, at most
+  int64_t nsched;             // work-list entries per pair, at most (key blocks + groups)
   int nvar, ntile, nsplit_max;
 };
 
@@ -147,15 +156,28 @@ vs_status run_recall_hist_dca(vs_ctx* c, const uint16_t* q, int64_t q_rows, int6
 vs_status run_recall_hist(vs_ctx* c, int64_t e, int nr, const float* lse, int nlev,
                           cudaStream_t st);
 // select.cu
-vs_status run_thresholds(vs_ctx* c, const float* vert, const float* slash, int64_t e_ld, int64_t e,
-                         const int32_t* kv, const int32_t* ks, int nlev, cudaStream_t st);
-vs_status run_levels(vs_ctx* c, const float* vert, const float* slash, int64_t e_ld, int64_t e,
-                     int nlev, cudaStream_t st);
-vs_status run_compact(vs_ctx* c, int64_t e, const int32_t* level_of_head, int32_t* v_idx,
-                      int32_t cap_v, int32_t* v_cnt, int32_t* s_off, int32_t cap_s,
-                      int32_t* s_cnt, cudaStream_t st);
+constexpr int kSelMaxSegments = 64;  // segments (CTAs) per (head, array), at most
+// Scratch of the selection kernels (the context's workspace, or the no-alloc array).
+struct SelScratch {
+  uint32_t* thr;   // thresholds [hq][2][kMaxLevels][2] (key, how many equal keys to take)
+  uint8_t* lvl;    // per-element levels [hq][2][e_pad]
+  int64_t e_pad;
+  void* state;     // radix-select state [hq][2] (sel_state_bytes)
+  uint32_t* part;  // per-segment histograms and counts (sel_part_bytes)
+  int* err;        // device error word
+};
+size_t sel_state_bytes(int hq);
+size_t sel_part_bytes(int hq, int nslot);  // nslot: levels selected at once (1 for vs_select)
+// Thresholds and levels of nlev budget levels (thresholds_and_levels), and/or the index
+// lists of the chosen level per head (compact; choice nullptr: level 0).
+vs_status launch_select(const SelScratch& sc, int hq, const float* vert, const float* slash, int64_t e_ld,
+                        int64_t e, const int32_t* kv, const int32_t* ks, int nlev, const int32_t* choice,
+                        int32_t* v_idx, int32_t cap_v, int32_t* v_cnt, int32_t* s_off, int32_t cap_s,
+                        int32_t* s_cnt, bool thresholds_and_levels, bool compact, cudaStream_t st);
 vs_status run_refine_decide(vs_ctx* c, int64_t e, int nr, int nlev, float tau, int32_t* kv,
                             int32_t* ks, float* recall, cudaStream_t st);
+vs_status run_budgets_max(int hq, const int32_t* kv, const int32_t* ks, int32_t* kv_acc, int32_t* ks_acc,
+                          cudaStream_t st);
 // attn.cu
 vs_status run_sparse_prefill(vs_ctx* c, const uint16_t* q, int64_t q_rows, int64_t q_pos0,
                              int64_t e, const uint16_t* k, const uint16_t* v, int64_t kv_rows,

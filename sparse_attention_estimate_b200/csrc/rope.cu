@@ -93,8 +93,33 @@ vs_status launch_rope_rows(vs_ctx* c, const bf16* in, int64_t in_rows, int64_t i
   return launched("rope_rows_kernel launch");
 }
 
+// Guard of a reused rotated-key cache: re-rotates kKCheckRows rows spread over [0, valid)
+// of every KV head and compares them bit for bit with the cache; a difference (the
+// caller rewrote K under the same pointer without vs_context_reset) raises the device
+// error word. One block per sampled row, one thread per (head, rotary pair).
+constexpr int kKCheckRows = 8;
+constexpr int kDevErrKCache = 5;
+__global__ void kcache_check_kernel(const uint16_t* __restrict__ k, int64_t k_rows, const uint16_t* __restrict__ cache,
+                                    int64_t cache_rows, int64_t valid, int nheads, int mode, DcaParams dca,
+                                    const double* __restrict__ theta, int* err) {
+  const int64_t r = valid <= 1 ? 0 : (valid - 1) * blockIdx.x / (kKCheckRows - 1);
+  const int64_t p = mode == 1 ? dca_key_pos(r, dca) : r;
+  for (int w = threadIdx.x; w < nheads * kHalf; w += blockDim.x) {
+    const int h = w / kHalf, m = w % kHalf;
+    const uint16_t* x = k + (static_cast<int64_t>(h) * k_rows + r) * kD;
+    const uint16_t* y = cache + (static_cast<int64_t>(h) * cache_rows + r) * kD;
+    double sn, cs;
+    sincos(__dmul_rn(static_cast<double>(p), theta[m]), &sn, &cs);
+    const double x1 = bf16_bits_to_f64(x[m]), x2 = bf16_bits_to_f64(x[m + kHalf]);
+    const uint16_t y1 = f64_to_bf16_rne(__dsub_rn(__dmul_rn(x1, cs), __dmul_rn(x2, sn)));
+    const uint16_t y2 = f64_to_bf16_rne(__dadd_rn(__dmul_rn(x2, cs), __dmul_rn(x1, sn)));
+    if (y1 != y[m] || y2 != y[m + kHalf]) atomicCAS(err, 0, kDevErrKCache);
+  }
+}
+
 // Extends a rotated-key cache to rows [0, e). The cache is keyed on the source
-// pointer and its row count; rows already rotated are assumed unchanged.
+// pointer and its row count; rows already rotated are assumed unchanged, which a
+// sampled re-rotation checks on the device whenever the cache is reused.
 vs_status ensure_keys_rotated(vs_ctx* c, const uint16_t* k, int64_t k_rows, int64_t e, bool dca,
                               cudaStream_t st) {
   KCache& kc = dca ? c->kd : c->kc;
@@ -102,6 +127,14 @@ vs_status ensure_keys_rotated(vs_ctx* c, const uint16_t* k, int64_t k_rows, int6
     kc.src = k;
     kc.src_rows = k_rows;
     kc.valid = 0;
+  }
+  if (kc.valid > 0) {
+    kcache_check_kernel<<<kKCheckRows, 256, 0, st>>>(k, k_rows,
+                                                    reinterpret_cast<const uint16_t*>(c->ws + (dca ? c->L.k_dca : c->L.k_cont)),
+                                                    c->max_seq, kc.valid, c->cfg.hkv, dca ? 1 : 0, c->dca, c->theta,
+                                                    c->err);
+    vs_status s = launched("kcache_check_kernel launch");
+    if (s != VS_OK) return s;
   }
   if (e <= kc.valid) return VS_OK;
   bf16* dst = ws_ptr<bf16>(c, dca ? c->L.k_dca : c->L.k_cont);

@@ -10,20 +10,30 @@
 // ascending) is fixed, the selected sets are nested and one pass can assign each
 // column / offset the first level that selects it.
 //
-// Kernels (one 1024-thread CTA per (head, array)):
-//  thresholds_kernel  - radix select (four 8-bit digit passes over the fp32 bit
-//                       pattern, which orders non-negative floats) of the k_t-th
-//                       largest key for every level at once, plus how many
-//                       elements equal to that key are taken (lowest index first)
-//  levels_kernel      - ordered pass writing each element's first level (255: none)
-//  compact_kernel     - ordered pass writing the ascending index list of a level
-//  refine_decide_kernel - first level whose recall reaches tau (or saturation)
+// Every (head, array) is cut into segments, one CTA each (several per array, so
+// that the arrays of all heads fill the SMs); threads load 16 bytes at a time.
+//  radix select   the k_t-th largest key of every level at once, four 8-bit digit
+//                 passes over the fp32 bit pattern (which orders non-negative
+//                 floats): per pass a histogram kernel over the segments and a
+//                 decide kernel per (head, array) that fixes the digit; the state
+//                 between passes (prefixes, ranks, distinct prefixes) lives in the
+//                 workspace. The result: the threshold key of each level and how
+//                 many elements equal to it are taken (lowest index first).
+//  levels         each element's first level (255: none); the order of elements
+//                 equal to a threshold (by index) comes from per-segment counts.
+//  compact        the ascending index list of one level per head, segments placed
+//                 by their counts.
+//  refine_decide  first level whose recall reaches tau (or saturation).
+#include <algorithm>
+
 #include "internal.cuh"
 
 namespace vs {
 
 constexpr uint32_t kNoThreshold = 0xFFFFFFFFu;  // level with k = 0: selects nothing
 constexpr int kDevErrCap = 3;                    // an output list was longer than its cap
+constexpr int kSelThreads = 512;                 // threads of the segment kernels
+constexpr int kSelTile = 4 * kSelThreads;        // elements per tile: four per thread
 
 // Sort key of element j: fp32 bit pattern of a non-negative score (0 for
 // non-positive or NaN), +inf for slash offset 0, which is always selected.
@@ -32,9 +42,27 @@ __device__ __forceinline__ uint32_t sel_key(float x, int64_t j, int arr) {
   return (x > 0.0f) ? __float_as_uint(x) : 0u;
 }
 
-// Exclusive block-wide prefix sum of v (blockDim.x == 1024); *total gets the sum.
+// The four keys of elements j0 .. j0+3 of array x (keys of elements at or past `hi`
+// are 0, and such elements are reported invalid by the callers). vec: x is 16-byte
+// aligned at every multiple of 4.
+__device__ __forceinline__ void load_keys4(const float* x, int64_t j0, int64_t hi, int arr, bool vec,
+                                           uint32_t (&k)[4]) {
+  if (vec && j0 + 3 < hi) {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(x + j0));
+    k[0] = sel_key(v.x, j0, arr);
+    k[1] = sel_key(v.y, j0 + 1, arr);
+    k[2] = sel_key(v.z, j0 + 2, arr);
+    k[3] = sel_key(v.w, j0 + 3, arr);
+  } else {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) k[q] = j0 + q < hi ? sel_key(__ldg(x + j0 + q), j0 + q, arr) : 0u;
+  }
+}
+
+// Exclusive block-wide prefix sum of v over the CTA's threads (blockDim.x ==
+// kSelThreads); *total gets the sum. wsum: 32 ints of shared memory.
 __device__ __forceinline__ int block_excl_scan(int v, int* wsum, int* total) {
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
   int x = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -44,7 +72,7 @@ __device__ __forceinline__ int block_excl_scan(int v, int* wsum, int* total) {
   if (lane == 31) wsum[w] = x;
   __syncthreads();
   if (w == 0) {
-    int s = wsum[lane];
+    int s = lane < nw ? wsum[lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int y = __shfl_up_sync(0xffffffffu, s, o);
@@ -54,110 +82,156 @@ __device__ __forceinline__ int block_excl_scan(int v, int* wsum, int* total) {
   }
   __syncthreads();
   const int base = (w > 0) ? wsum[w - 1] : 0;
-  *total = wsum[31];
+  *total = wsum[nw - 1];
   __syncthreads();
   return base + x - v;
 }
 
-__global__ void __launch_bounds__(1024) thresholds_kernel(const float* __restrict__ vert,
-                                                          const float* __restrict__ slash,
-                                                          int64_t e_ld, int64_t e,
-                                                          const int32_t* __restrict__ kv,
-                                                          const int32_t* __restrict__ ks, int nlev,
-                                                          uint32_t* __restrict__ thr) {
-  const int h = blockIdx.x, arr = blockIdx.y, tid = threadIdx.x;
-  const float* x = (arr == 0 ? vert : slash) + static_cast<int64_t>(h) * e_ld;
-  __shared__ uint32_t hist[kMaxLevels][256];
-  __shared__ uint32_t prefix[kMaxLevels], uprefix[kMaxLevels];
-  __shared__ int64_t rank[kMaxLevels];
-  __shared__ int slot_of[kMaxLevels], active[kMaxLevels];
-  __shared__ int nuniq;
-  if (tid < nlev) {
+// Radix-select state of one (head, array) between passes.
+struct RadixState {
+  uint32_t prefix[kMaxLevels];   // digits of the level's threshold fixed so far
+  uint32_t uprefix[kMaxLevels];  // distinct prefixes of the active levels
+  int32_t slot[kMaxLevels];      // the level's entry in uprefix (-1: inactive level)
+  int32_t nu;                    // distinct prefixes
+  int32_t pad;
+  long long rank[kMaxLevels];    // rank still to find among the elements with the prefix
+};
+
+__device__ __forceinline__ const float* sel_row(const float* vert, const float* slash, int64_t e_ld, int h,
+                                                int arr) {
+  return (arr == 0 ? vert : slash) + static_cast<int64_t>(h) * e_ld;
+}
+
+// Level budgets k_t = min(base * 2^t, e) (base <= 0: the level selects nothing); all
+// active levels start with the empty prefix.
+__global__ void radix_init_kernel(const int32_t* __restrict__ kv, const int32_t* __restrict__ ks, int64_t e,
+                                  int nlev, RadixState* __restrict__ rs) {
+  const int h = blockIdx.y, arr = blockIdx.x, t = threadIdx.x;
+  RadixState& st = rs[h * 2 + arr];
+  __shared__ int any;
+  if (t == 0) any = 0;
+  __syncthreads();
+  if (t < kMaxLevels) {
     int64_t base = (arr == 0) ? kv[h] : ks[h];
     if (base < 0) base = 0;
-    int64_t k = base << tid;
-    if (k > e || (tid > 0 && (base << (tid - 1)) >= e)) k = e;
-    if (base == 0) k = 0;
-    rank[tid] = k;
-    prefix[tid] = 0;
-    active[tid] = k > 0;
+    int64_t k = 0;
+    if (t < nlev && base > 0) {
+      k = (t < 40 && base <= (e >> t)) ? (base << t) : e;
+      if (k > e) k = e;
+    }
+    st.prefix[t] = 0;
+    st.rank[t] = k;
+    st.slot[t] = k > 0 ? 0 : -1;
+    if (k > 0) atomicOr(&any, 1);
   }
   __syncthreads();
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    if (tid == 0) {
-      int nu = 0;
-      for (int t = 0; t < nlev; ++t) {
-        slot_of[t] = -1;
-        if (!active[t]) continue;
-        int u = 0;
-        while (u < nu && uprefix[u] != prefix[t]) ++u;
-        if (u == nu) uprefix[nu++] = prefix[t];
-        slot_of[t] = u;
-      }
-      nuniq = nu;
-    }
-    __syncthreads();
-    const int nu = nuniq;
-    for (int i = tid; i < nu * 256; i += blockDim.x) (&hist[0][0])[i] = 0;
-    __syncthreads();
-    for (int64_t j0 = 0; j0 < e; j0 += blockDim.x) {
-      const int64_t j = j0 + tid;
-      int u = -1;
-      uint32_t digit = 0;
-      if (j < e) {
-        const uint32_t key = sel_key(x[j], j, arr);
-        const uint32_t hp = (pass == 0) ? 0u : (key >> (shift + 8));
-        for (int uu = 0; uu < nu; ++uu)
-          if (uprefix[uu] == hp) {
-            u = uu;
-            break;
-          }
-        digit = (key >> shift) & 255u;
-      }
-      // aggregate equal (slot, digit) pairs of the warp into one atomic
-      const uint32_t tag = (u < 0) ? 0xFFFFFFFFu : ((static_cast<uint32_t>(u) << 8) | digit);
-      const uint32_t peers = __match_any_sync(0xffffffffu, tag);
-      if (u >= 0 && (__ffs(peers) - 1) == (tid & 31))
-        atomicAdd(&hist[u][digit], static_cast<uint32_t>(__popc(peers)));
-    }
-    __syncthreads();
-    if (tid < nlev && active[tid]) {
-      const int u = slot_of[tid];
-      int64_t cum = 0;
-      for (int d = 255; d >= 0; --d) {
-        const int64_t cnt = hist[u][d];
-        if (cum + cnt >= rank[tid]) {
-          prefix[tid] = (prefix[tid] << 8) | static_cast<uint32_t>(d);
-          rank[tid] -= cum;
-          break;
-        }
-        cum += cnt;
-      }
-    }
-    __syncthreads();
-  }
-  if (tid < kMaxLevels) {
-    uint32_t* o = thr + ((static_cast<int64_t>(h) * 2 + arr) * kMaxLevels + tid) * 2;
-    const bool ok = tid < nlev && active[tid];
-    o[0] = ok ? prefix[tid] : kNoThreshold;
-    o[1] = ok ? static_cast<uint32_t>(rank[tid]) : 0u;
+  if (t == 0) {
+    st.uprefix[0] = 0;
+    st.nu = any ? 1 : 0;
   }
 }
 
-__global__ void __launch_bounds__(1024) levels_kernel(const float* __restrict__ vert,
-                                                      const float* __restrict__ slash, int64_t e_ld,
-                                                      int64_t e, int nlev,
-                                                      const uint32_t* __restrict__ thr,
-                                                      uint8_t* __restrict__ lvl, int64_t e_pad) {
-  const int h = blockIdx.x, arr = blockIdx.y, tid = threadIdx.x;
-  const float* x = (arr == 0 ? vert : slash) + static_cast<int64_t>(h) * e_ld;
-  uint8_t* out = lvl + (static_cast<int64_t>(h) * 2 + arr) * e_pad;
-  __shared__ uint32_t T[kMaxLevels], take[kMaxLevels], uT[kMaxLevels];
-  __shared__ int64_t run[kMaxLevels];
+// One digit pass: histograms of digit (key >> shift) & 255 of the segment's elements,
+// per distinct prefix (the key's bits above the digit), into part[(h,arr,seg)][slot][256].
+__global__ void __launch_bounds__(kSelThreads) radix_hist_kernel(
+    const float* __restrict__ vert, const float* __restrict__ slash, int64_t e_ld, int64_t e, int64_t seg,
+    bool vec, int shift, const RadixState* __restrict__ rs, uint32_t* __restrict__ part, int nslot) {
+  const int b = blockIdx.x, arr = blockIdx.y, h = blockIdx.z, tid = threadIdx.x;
+  const RadixState& st = rs[h * 2 + arr];
+  const int nu = st.nu;
+  if (nu == 0) return;
+  extern __shared__ uint32_t hist[];  // [nu][256]
+  __shared__ uint32_t up[kMaxLevels];
+  for (int i = tid; i < nu * 256; i += blockDim.x) hist[i] = 0u;
+  if (tid < nu) up[tid] = st.uprefix[tid];
+  __syncthreads();
+  const float* x = sel_row(vert, slash, e_ld, h, arr);
+  const int64_t lo = static_cast<int64_t>(b) * seg, hi = min(lo + seg, e);
+  for (int64_t t0 = lo; t0 < hi; t0 += kSelTile) {  // the same trip count for every thread
+    const int64_t j0 = t0 + 4 * tid;
+    uint32_t k[4];
+    load_keys4(x, j0, hi, arr, vec, k);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      int u = -1;
+      uint32_t digit = 0;
+      if (j0 + q < hi) {
+        const uint32_t hp = shift == 24 ? 0u : (k[q] >> (shift + 8));
+        for (int uu = 0; uu < nu; ++uu)
+          if (up[uu] == hp) {
+            u = uu;
+            break;
+          }
+        digit = (k[q] >> shift) & 255u;
+      }
+      // equal (prefix, digit) pairs of the warp add once
+      const uint32_t tag = u < 0 ? 0xFFFFFFFFu : ((static_cast<uint32_t>(u) << 8) | digit);
+      const uint32_t peers = __match_any_sync(0xffffffffu, tag);
+      if (u >= 0 && (__ffs(peers) - 1) == (tid & 31)) atomicAdd(&hist[u * 256 + digit], __popc(peers));
+    }
+  }
+  __syncthreads();
+  uint32_t* o = part + (static_cast<int64_t>(h * 2 + arr) * gridDim.x + b) * nslot * 256;
+  for (int i = tid; i < nu * 256; i += blockDim.x) o[i] = hist[i];
+}
+
+// Fixes one digit of every active level from the segments' histograms; after the last
+// pass (final) writes the thresholds thr[(h,arr)][t] = (key, how many equal keys to take).
+__global__ void __launch_bounds__(256) radix_decide_kernel(RadixState* __restrict__ rs,
+                                                           const uint32_t* __restrict__ part, int nseg,
+                                                           int nslot, bool final, int nlev,
+                                                           uint32_t* __restrict__ thr) {
+  const int arr = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+  RadixState& st = rs[h * 2 + arr];
+  const int nu = st.nu;
+  __shared__ uint32_t hist[kMaxLevels][256];
+  const uint32_t* pp = part + static_cast<int64_t>(h * 2 + arr) * nseg * nslot * 256;
+  for (int u = 0; u < nu; ++u) {
+    uint32_t sum = 0;
+    for (int b = 0; b < nseg; ++b) sum += pp[(static_cast<int64_t>(b) * nslot + u) * 256 + tid];
+    hist[u][tid] = sum;
+  }
+  __syncthreads();
+  if (tid < kMaxLevels && st.slot[tid] >= 0) {
+    const int u = st.slot[tid];
+    long long cum = 0;
+    const long long r = st.rank[tid];
+    for (int d = 255; d >= 0; --d) {
+      const long long cnt = hist[u][d];
+      if (cum + cnt >= r) {
+        st.prefix[tid] = (st.prefix[tid] << 8) | static_cast<uint32_t>(d);
+        st.rank[tid] = r - cum;
+        break;
+      }
+      cum += cnt;
+    }
+  }
+  __syncthreads();
+  if (tid == 0) {  // distinct prefixes of the active levels, for the next pass
+    int n = 0;
+    for (int t = 0; t < kMaxLevels; ++t) {
+      if (st.slot[t] < 0) continue;
+      int u = 0;
+      while (u < n && st.uprefix[u] != st.prefix[t]) ++u;
+      if (u == n) st.uprefix[n++] = st.prefix[t];
+      st.slot[t] = u;
+    }
+    st.nu = n;
+  }
+  __syncthreads();
+  if (final && tid < kMaxLevels) {
+    uint32_t* o = thr + (static_cast<int64_t>(h) * 2 + arr) * kMaxLevels * 2 + 2 * tid;
+    const bool ok = tid < nlev && st.slot[tid] >= 0;
+    o[0] = ok ? st.prefix[tid] : kNoThreshold;
+    o[1] = ok ? static_cast<uint32_t>(st.rank[tid]) : 0u;
+  }
+}
+
+// The distinct threshold keys of one (head, array) into shared memory; returns how many.
+__device__ __forceinline__ int load_thresholds(const uint32_t* thr, int h, int arr, int nlev, uint32_t* T,
+                                               uint32_t* take, uint32_t* uT) {
   __shared__ int nu_s;
-  __shared__ int wsum[32];
-  if (tid == 0) {
+  if (threadIdx.x == 0) {
     int nu = 0;
     for (int t = 0; t < nlev; ++t) {
       const uint32_t* p = thr + ((static_cast<int64_t>(h) * 2 + arr) * kMaxLevels + t) * 2;
@@ -166,78 +240,191 @@ __global__ void __launch_bounds__(1024) levels_kernel(const float* __restrict__ 
       if (p[0] == kNoThreshold) continue;
       int u = 0;
       while (u < nu && uT[u] != p[0]) ++u;
-      if (u == nu) {
-        uT[nu] = p[0];
-        run[nu] = 0;
-        ++nu;
-      }
+      if (u == nu) uT[nu++] = p[0];
     }
     nu_s = nu;
   }
   __syncthreads();
-  const int nu = nu_s;
-  for (int64_t j0 = 0; j0 < e; j0 += blockDim.x) {
-    const int64_t j = j0 + tid;
-    const bool valid = j < e;
-    const uint32_t key = valid ? sel_key(x[j], j, arr) : 0u;
-    int myu = -1;
-    if (valid)
-      for (int u = 0; u < nu; ++u)
-        if (uT[u] == key) {
-          myu = u;
-          break;
-        }
-    int64_t myrank = 0;
-    if (__syncthreads_or(myu >= 0)) {
+  return nu_s;
+}
+
+// Per segment: how many elements equal each distinct threshold key, into
+// cnt[(h,arr,seg)][u].
+__global__ void __launch_bounds__(kSelThreads) eq_count_kernel(
+    const float* __restrict__ vert, const float* __restrict__ slash, int64_t e_ld, int64_t e, int64_t seg,
+    bool vec, int nlev, const uint32_t* __restrict__ thr, int32_t* __restrict__ cnt) {
+  const int b = blockIdx.x, arr = blockIdx.y, h = blockIdx.z, tid = threadIdx.x;
+  __shared__ uint32_t T[kMaxLevels], take[kMaxLevels], uT[kMaxLevels];
+  __shared__ int c_s[kMaxLevels];
+  if (tid < kMaxLevels) c_s[tid] = 0;
+  const int nu = load_thresholds(thr, h, arr, nlev, T, take, uT);
+  const float* x = sel_row(vert, slash, e_ld, h, arr);
+  const int64_t lo = static_cast<int64_t>(b) * seg, hi = min(lo + seg, e);
+  for (int64_t t0 = lo; t0 < hi; t0 += kSelTile) {
+    const int64_t j0 = t0 + 4 * tid;
+    uint32_t k[4];
+    load_keys4(x, j0, hi, arr, vec, k);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (j0 + q < hi)
+        for (int u = 0; u < nu; ++u)
+          if (k[q] == uT[u]) {
+            atomicAdd(&c_s[u], 1);
+            break;
+          }
+  }
+  __syncthreads();
+  if (tid < kMaxLevels) cnt[(static_cast<int64_t>(h * 2 + arr) * gridDim.x + b) * kMaxLevels + tid] = c_s[tid];
+}
+
+// Each element's first level: key above the level's threshold, or equal to it and among
+// the first `take` such elements by index (255: no level selects it).
+__global__ void __launch_bounds__(kSelThreads) levels_kernel(
+    const float* __restrict__ vert, const float* __restrict__ slash, int64_t e_ld, int64_t e, int64_t seg,
+    bool vec, int nlev, const uint32_t* __restrict__ thr, const int32_t* __restrict__ cnt,
+    uint8_t* __restrict__ lvl, int64_t e_pad) {
+  const int b = blockIdx.x, arr = blockIdx.y, h = blockIdx.z, tid = threadIdx.x;
+  __shared__ uint32_t T[kMaxLevels], take[kMaxLevels], uT[kMaxLevels];
+  __shared__ long long run[kMaxLevels];
+  __shared__ int wsum[32];
+  const int nu = load_thresholds(thr, h, arr, nlev, T, take, uT);
+  if (tid < nu) {  // equal keys in the earlier segments
+    long long r = 0;
+    for (int bb = 0; bb < b; ++bb) r += cnt[(static_cast<int64_t>(h * 2 + arr) * gridDim.x + bb) * kMaxLevels + tid];
+    run[tid] = r;
+  }
+  __syncthreads();
+  const float* x = sel_row(vert, slash, e_ld, h, arr);
+  uint8_t* out = lvl + (static_cast<int64_t>(h) * 2 + arr) * e_pad;
+  const int64_t lo = static_cast<int64_t>(b) * seg, hi = min(lo + seg, e);
+  for (int64_t t0 = lo; t0 < hi; t0 += kSelTile) {
+    const int64_t j0 = t0 + 4 * tid;
+    uint32_t k[4];
+    load_keys4(x, j0, hi, arr, vec, k);
+    int myu[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      myu[q] = -1;
+      if (j0 + q < hi)
+        for (int u = 0; u < nu; ++u)
+          if (k[q] == uT[u]) {
+            myu[q] = u;
+            break;
+          }
+    }
+    long long rk[4] = {0, 0, 0, 0};
+    const bool mine = myu[0] >= 0 || myu[1] >= 0 || myu[2] >= 0 || myu[3] >= 0;
+    if (__syncthreads_or(mine)) {
       for (int u = 0; u < nu; ++u) {
-        if (!__syncthreads_or(myu == u)) continue;
+        const int c = (myu[0] == u) + (myu[1] == u) + (myu[2] == u) + (myu[3] == u);
+        if (!__syncthreads_or(c > 0)) continue;
         int total = 0;
-        const int r = block_excl_scan(myu == u ? 1 : 0, wsum, &total);
-        if (myu == u) myrank = run[u] + r;
+        int r = block_excl_scan(c, wsum, &total);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (myu[q] == u) rk[q] = run[u] + r++;
         __syncthreads();
         if (tid == 0) run[u] += total;
         __syncthreads();
       }
     }
-    if (valid) {
-      uint8_t level = 255;
-      for (int t = 0; t < nlev; ++t) {
-        const uint32_t tt = T[t];
-        if (tt == kNoThreshold) continue;
-        if (key > tt || (key == tt && myrank < static_cast<int64_t>(take[t]))) {
-          level = static_cast<uint8_t>(t);
-          break;
+    uint32_t packed = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t level = 255;
+      if (j0 + q < hi)
+        for (int t = 0; t < nlev; ++t) {
+          const uint32_t tt = T[t];
+          if (tt == kNoThreshold) continue;
+          if (k[q] > tt || (k[q] == tt && rk[q] < static_cast<long long>(take[t]))) {
+            level = static_cast<uint32_t>(t);
+            break;
+          }
         }
-      }
-      out[j] = level;
+      packed |= level << (8 * q);
     }
+    if (j0 + 3 < hi)
+      *reinterpret_cast<uint32_t*>(out + j0) = packed;  // j0 % 4 == 0, rows 128-aligned
+    else
+      for (int q = 0; q < 4; ++q)
+        if (j0 + q < hi) out[j0 + q] = static_cast<uint8_t>(packed >> (8 * q));
   }
 }
 
-__global__ void __launch_bounds__(1024) compact_kernel(const uint8_t* __restrict__ lvl,
-                                                       int64_t e_pad, int64_t e,
-                                                       const int32_t* __restrict__ choice,
-                                                       int32_t* v_idx, int32_t cap_v,
-                                                       int32_t* v_cnt, int32_t* s_off,
-                                                       int32_t cap_s, int32_t* s_cnt, int* err) {
-  const int h = blockIdx.x, arr = blockIdx.y, tid = threadIdx.x;
+// The four level bytes of elements j0 .. j0+3 that are at or below level tsel.
+__device__ __forceinline__ int selected4(const uint8_t* lv, int64_t j0, int64_t hi, int tsel, bool (&f)[4]) {
+  uint32_t w4 = 0xFFFFFFFFu;
+  if (j0 + 3 < hi)
+    w4 = *reinterpret_cast<const uint32_t*>(lv + j0);
+  else
+    for (int q = 0; q < 4; ++q)
+      if (j0 + q < hi) w4 = (w4 & ~(0xFFu << (8 * q))) | (static_cast<uint32_t>(lv[j0 + q]) << (8 * q));
+  int c = 0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    f[q] = static_cast<int>((w4 >> (8 * q)) & 0xFFu) <= tsel;
+    c += f[q];
+  }
+  return c;
+}
+
+// Per segment: elements selected at the head's chosen level (level 0 without a choice).
+__global__ void __launch_bounds__(kSelThreads) compact_count_kernel(const uint8_t* __restrict__ lvl,
+                                                                    int64_t e_pad, int64_t e, int64_t seg,
+                                                                    const int32_t* __restrict__ choice,
+                                                                    int32_t* __restrict__ cnt) {
+  const int b = blockIdx.x, arr = blockIdx.y, h = blockIdx.z, tid = threadIdx.x;
+  const uint8_t* lv = lvl + (static_cast<int64_t>(h) * 2 + arr) * e_pad;
+  const int tsel = choice ? choice[h] : 0;
+  const int64_t lo = static_cast<int64_t>(b) * seg, hi = min(lo + seg, e);
+  int c = 0;
+  for (int64_t t0 = lo; t0 < hi; t0 += kSelTile) {
+    bool f[4];
+    c += selected4(lv, t0 + 4 * tid, hi, tsel, f);
+  }
+  __shared__ int wsum[32];
+  int total = 0;
+  block_excl_scan(c, wsum, &total);
+  if (tid == 0) cnt[static_cast<int64_t>(h * 2 + arr) * gridDim.x + b] = total;
+}
+
+// The ascending index list of the selected elements: the segment's elements go after
+// those of the earlier segments. The last segment's CTA writes the list length.
+__global__ void __launch_bounds__(kSelThreads) compact_write_kernel(
+    const uint8_t* __restrict__ lvl, int64_t e_pad, int64_t e, int64_t seg, const int32_t* __restrict__ choice,
+    const int32_t* __restrict__ cnt, int32_t* v_idx, int32_t cap_v, int32_t* v_cnt, int32_t* s_off,
+    int32_t cap_s, int32_t* s_cnt, int* err) {
+  const int b = blockIdx.x, arr = blockIdx.y, h = blockIdx.z, tid = threadIdx.x;
   const uint8_t* lv = lvl + (static_cast<int64_t>(h) * 2 + arr) * e_pad;
   const int tsel = choice ? choice[h] : 0;
   const int32_t cap = arr == 0 ? cap_v : cap_s;
-  int32_t* out = arr == 0 ? v_idx + static_cast<int64_t>(h) * cap_v
-                          : s_off + static_cast<int64_t>(h) * cap_s;
+  int32_t* out = arr == 0 ? v_idx + static_cast<int64_t>(h) * cap_v : s_off + static_cast<int64_t>(h) * cap_s;
+  const int32_t* cc = cnt + static_cast<int64_t>(h * 2 + arr) * gridDim.x;
   __shared__ int wsum[32];
-  int64_t running = 0;
-  for (int64_t j0 = 0; j0 < e; j0 += blockDim.x) {
-    const int64_t j = j0 + tid;
-    const int flag = (j < e && static_cast<int>(lv[j]) <= tsel) ? 1 : 0;
+  __shared__ long long base_s;
+  if (tid == 0) {
+    long long r = 0;
+    for (int bb = 0; bb < b; ++bb) r += cc[bb];
+    base_s = r;
+  }
+  __syncthreads();
+  long long running = base_s;
+  const int64_t lo = static_cast<int64_t>(b) * seg, hi = min(lo + seg, e);
+  for (int64_t t0 = lo; t0 < hi; t0 += kSelTile) {
+    const int64_t j0 = t0 + 4 * tid;
+    bool f[4];
+    const int c = selected4(lv, j0, hi, tsel, f);
     int total = 0;
-    const int r = block_excl_scan(flag, wsum, &total);
-    const int64_t pos = running + r;
-    if (flag && pos < cap) out[pos] = static_cast<int32_t>(j);
+    long long pos = running + block_excl_scan(c, wsum, &total);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (f[q]) {
+        if (pos < cap) out[pos] = static_cast<int32_t>(j0 + q);
+        ++pos;
+      }
     running += total;
   }
-  if (tid == 0) {
+  if (b == static_cast<int>(gridDim.x) - 1 && tid == 0) {
     (arr == 0 ? v_cnt : s_cnt)[h] = static_cast<int32_t>(running < cap ? running : cap);
     if (running > cap) atomicCAS(err, 0, kDevErrCap);
   }
@@ -274,28 +461,19 @@ __global__ void refine_decide_kernel(const float* __restrict__ hist, int nsplit,
   recall[h] = static_cast<float>(rc);
 }
 
-vs_status run_thresholds(vs_ctx* c, const float* vert, const float* slash, int64_t e_ld, int64_t e,
-                         const int32_t* kv, const int32_t* ks, int nlev, cudaStream_t st) {
-  thresholds_kernel<<<dim3(c->cfg.hq, 2), 1024, 0, st>>>(vert, slash, e_ld, e, kv, ks, nlev,
-                                                        ws_ptr<uint32_t>(c, c->L.thr));
-  return launched("thresholds_kernel launch");
+// Offline calibration: acc[h] = max(acc[h], budget[h]) for both budgets.
+__global__ void budgets_max_kernel(int hq, const int32_t* __restrict__ kv, const int32_t* __restrict__ ks,
+                                   int32_t* kv_acc, int32_t* ks_acc) {
+  const int h = blockIdx.x * blockDim.x + threadIdx.x;
+  if (h >= hq) return;
+  kv_acc[h] = max(kv_acc[h], kv[h]);
+  ks_acc[h] = max(ks_acc[h], ks[h]);
 }
 
-vs_status run_levels(vs_ctx* c, const float* vert, const float* slash, int64_t e_ld, int64_t e,
-                     int nlev, cudaStream_t st) {
-  levels_kernel<<<dim3(c->cfg.hq, 2), 1024, 0, st>>>(vert, slash, e_ld, e, nlev,
-                                                    ws_ptr<uint32_t>(c, c->L.thr),
-                                                    ws_ptr<uint8_t>(c, c->L.lvl), c->L.e_pad);
-  return launched("levels_kernel launch");
-}
-
-vs_status run_compact(vs_ctx* c, int64_t e, const int32_t* level_of_head, int32_t* v_idx,
-                      int32_t cap_v, int32_t* v_cnt, int32_t* s_off, int32_t cap_s,
-                      int32_t* s_cnt, cudaStream_t st) {
-  compact_kernel<<<dim3(c->cfg.hq, 2), 1024, 0, st>>>(ws_ptr<uint8_t>(c, c->L.lvl), c->L.e_pad, e,
-                                                     level_of_head, v_idx, cap_v, v_cnt, s_off,
-                                                     cap_s, s_cnt, c->err);
-  return launched("compact_kernel launch");
+vs_status run_budgets_max(int hq, const int32_t* kv, const int32_t* ks, int32_t* kv_acc, int32_t* ks_acc,
+                          cudaStream_t st) {
+  budgets_max_kernel<<<static_cast<unsigned>(ceil_div(hq, 128)), 128, 0, st>>>(hq, kv, ks, kv_acc, ks_acc);
+  return launched("budgets_max_kernel launch");
 }
 
 vs_status run_refine_decide(vs_ctx* c, int64_t e, int nr, int nlev, float tau, int32_t* kv,
@@ -306,21 +484,69 @@ vs_status run_refine_decide(vs_ctx* c, int64_t e, int nr, int nlev, float tau, i
   return launched("refine_decide_kernel launch");
 }
 
-// The three selection kernels on caller-given scratch pointers (no context):
-// thr [hq][2][kMaxLevels][2] uint32, lvl [hq][2][e_pad] uint8, err one int.
-vs_status launch_select_raw(int hq, const float* vert, const float* slash, int64_t e_ld, int64_t e,
-                            const int32_t* kv, const int32_t* ks, uint32_t* thr, uint8_t* lvl,
-                            int64_t e_pad, int* err, int32_t* v_idx, int32_t cap_v, int32_t* v_cnt,
-                            int32_t* s_off, int32_t cap_s, int32_t* s_cnt, cudaStream_t st) {
-  thresholds_kernel<<<dim3(hq, 2), 1024, 0, st>>>(vert, slash, e_ld, e, kv, ks, 1, thr);
-  vs_status s = launched("thresholds_kernel launch");
-  if (s != VS_OK) return s;
-  levels_kernel<<<dim3(hq, 2), 1024, 0, st>>>(vert, slash, e_ld, e, 1, thr, lvl, e_pad);
-  s = launched("levels_kernel launch");
-  if (s != VS_OK) return s;
-  compact_kernel<<<dim3(hq, 2), 1024, 0, st>>>(lvl, e_pad, e, nullptr, v_idx, cap_v, v_cnt, s_off,
-                                              cap_s, s_cnt, err);
-  return launched("compact_kernel launch");
+
+// Segments per (head, array): enough CTAs over all heads to fill the SMs about four
+// times, each segment at least one tile and a multiple of the tile.
+int select_max_segments(int hq);
+int select_segments(int hq, int64_t e, int64_t* seg_out) {
+  int nseg = select_max_segments(hq);
+  nseg = static_cast<int>(std::min<int64_t>(nseg, ceil_div(e, kSelTile)));
+  nseg = std::max(1, nseg);
+  const int64_t seg = round_up(ceil_div(e, nseg), kSelTile);
+  *seg_out = seg;
+  return static_cast<int>(ceil_div(e, seg));
+}
+
+vs_status launch_select(const SelScratch& sc, int hq, const float* vert, const float* slash, int64_t e_ld,
+                        int64_t e, const int32_t* kv, const int32_t* ks, int nlev, const int32_t* choice,
+                        int32_t* v_idx, int32_t cap_v, int32_t* v_cnt, int32_t* s_off, int32_t cap_s,
+                        int32_t* s_cnt, bool thresholds_and_levels, bool compact, cudaStream_t st) {
+  int64_t seg = 0;
+  const int nseg = select_segments(hq, e, &seg);
+  const bool vec = (e_ld % 4) == 0 && (reinterpret_cast<uintptr_t>(vert) & 15u) == 0 &&
+                   (reinterpret_cast<uintptr_t>(slash) & 15u) == 0;
+  const dim3 grid(nseg, 2, hq);
+  vs_status s = VS_OK;
+  if (thresholds_and_levels) {
+    RadixState* rs = reinterpret_cast<RadixState*>(sc.state);
+    radix_init_kernel<<<dim3(2, hq), 32, 0, st>>>(kv, ks, e, nlev, rs);
+    s = launched("radix_init_kernel launch");
+    for (int pass = 0; pass < 4 && s == VS_OK; ++pass) {
+      radix_hist_kernel<<<grid, kSelThreads, nlev * 256 * sizeof(uint32_t), st>>>(
+          vert, slash, e_ld, e, seg, vec, 24 - 8 * pass, rs, sc.part, nlev);
+      s = launched("radix_hist_kernel launch");
+      if (s != VS_OK) break;
+      radix_decide_kernel<<<dim3(2, hq), 256, 0, st>>>(rs, sc.part, nseg, nlev, pass == 3, nlev, sc.thr);
+      s = launched("radix_decide_kernel launch");
+    }
+    if (s != VS_OK) return s;
+    int32_t* cnt = reinterpret_cast<int32_t*>(sc.part);  // the histograms are consumed
+    eq_count_kernel<<<grid, kSelThreads, 0, st>>>(vert, slash, e_ld, e, seg, vec, nlev, sc.thr, cnt);
+    s = launched("eq_count_kernel launch");
+    if (s != VS_OK) return s;
+    levels_kernel<<<grid, kSelThreads, 0, st>>>(vert, slash, e_ld, e, seg, vec, nlev, sc.thr, cnt, sc.lvl,
+                                                sc.e_pad);
+    s = launched("levels_kernel launch");
+    if (s != VS_OK) return s;
+  }
+  if (compact) {
+    int32_t* cnt = reinterpret_cast<int32_t*>(sc.part);
+    compact_count_kernel<<<grid, kSelThreads, 0, st>>>(sc.lvl, sc.e_pad, e, seg, choice, cnt);
+    s = launched("compact_count_kernel launch");
+    if (s != VS_OK) return s;
+    compact_write_kernel<<<grid, kSelThreads, 0, st>>>(sc.lvl, sc.e_pad, e, seg, choice, cnt, v_idx, cap_v,
+                                                       v_cnt, s_off, cap_s, s_cnt, sc.err);
+    s = launched("compact_write_kernel launch");
+  }
+  return s;
+}
+
+int select_max_segments(int hq) {
+  return std::max(1, std::min(static_cast<int>(ceil_div(4 * 148, 2 * hq)), kSelMaxSegments));
+}
+size_t sel_state_bytes(int hq) { return static_cast<size_t>(hq) * 2 * sizeof(RadixState); }
+size_t sel_part_bytes(int hq, int nslot) {
+  return static_cast<size_t>(hq) * 2 * select_max_segments(hq) * nslot * 256 * sizeof(uint32_t);
 }
 
 }  // namespace vs

@@ -36,10 +36,6 @@ constexpr int kNoAllocMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_select_scratch[kNoAllocScratchBytes];
 
-vs_status launch_select_raw(int hq, const float* vert, const float* slash, int64_t e_ld, int64_t e,
-                            const int32_t* kv, const int32_t* ks, uint32_t* thr, uint8_t* lvl,
-                            int64_t e_pad, int* err, int32_t* v_idx, int32_t cap_v, int32_t* v_cnt,
-                            int32_t* s_off, int32_t cap_s, int32_t* s_cnt, cudaStream_t st);
 
 // Driver calls through the runtime's driver entry point (no link against libcuda).
 template <class Fn>
@@ -110,12 +106,15 @@ extern "C" vs_status vs_select_noalloc(int32_t hq, const float* vert, const floa
   if (e < 1 || e_ld < e) return set_error(VS_ERR_INVALID_ARG, "need 1 <= e <= e_ld");
   if (cap_v < e || cap_s < e)
     return set_error(VS_ERR_INVALID_ARG, "caps must hold e entries (cap_v, cap_s >= e)");
-  // scratch: thresholds, one error word, per-element levels of both arrays
+  // scratch: thresholds, one error word, radix-select state, per-segment histograms,
+  // per-element levels of both arrays
   const int64_t e_pad = round_up(e, kTile);
   const size_t thr_bytes = round_up(static_cast<int64_t>(hq) * 2 * kMaxLevels * 2 * 4, 256);
   const size_t err_bytes = 256;
+  const size_t state_bytes = round_up(static_cast<int64_t>(sel_state_bytes(hq)), 256);
+  const size_t part_bytes = round_up(static_cast<int64_t>(sel_part_bytes(hq, 1)), 256);
   const size_t lvl_bytes = static_cast<size_t>(hq) * 2 * static_cast<size_t>(e_pad);
-  const size_t need = thr_bytes + err_bytes + lvl_bytes;
+  const size_t need = thr_bytes + err_bytes + state_bytes + part_bytes + lvl_bytes;
   if (need > kNoAllocScratchBytes)
     return set_error(VS_ERR_UNSUPPORTED,
                      "hq=%d, e=%lld needs %zu bytes of selection scratch; the no-alloc scratch "
@@ -124,8 +123,18 @@ extern "C" vs_status vs_select_noalloc(int32_t hq, const float* vert, const floa
   unsigned char* base = nullptr;
   vs_status s = scratch_address(&base);
   if (s != VS_OK) return s;
-  return launch_select_raw(hq, vert, slash, e_ld, e, kv_budget, ks_budget,
-                           reinterpret_cast<uint32_t*>(base), base + thr_bytes + err_bytes, e_pad,
-                           reinterpret_cast<int*>(base + thr_bytes), v_idx, cap_v, v_cnt, s_off,
-                           cap_s, s_cnt, stream);
+  unsigned char* p = base;
+  SelScratch sc{};
+  sc.thr = reinterpret_cast<uint32_t*>(p);
+  p += thr_bytes;
+  sc.err = reinterpret_cast<int*>(p);
+  p += err_bytes;
+  sc.state = p;
+  p += state_bytes;
+  sc.part = reinterpret_cast<uint32_t*>(p);
+  p += part_bytes;
+  sc.lvl = p;
+  sc.e_pad = e_pad;
+  return launch_select(sc, hq, vert, slash, e_ld, e, kv_budget, ks_budget, 1, nullptr, v_idx, cap_v, v_cnt,
+                       s_off, cap_s, s_cnt, true, true, stream);
 }

@@ -62,9 +62,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 
 // Waits for the phase with the given parity to complete. Returns false when the
 // CTA is aborting (abort word set by another thread) or the wait ran out; in the
-// latter case it raises the abort word and the device error word.
+// latter case it raises the abort word and the device error word, and the first
+// wait to run out records where it was: dev_err[1] = site + 256 * warp + 65536 *
+// CTA, dev_err[2] = `pos` (e.g. the work-list position).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_word,
-                                          int* dev_err) {
+                                          int* dev_err, int site = 0, int pos = 0) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
@@ -74,7 +76,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (*abort_word) return false;
     if (globaltimer_ns() - t0 > kWaitLimitNs) {
       *abort_word = 1;
-      if (dev_err) atomicCAS(dev_err, 0, kDevErrTimeout);
+      if (dev_err && atomicCAS(dev_err, 0, kDevErrTimeout) == 0) {
+        dev_err[1] = site + 256 * static_cast<int>(threadIdx.x >> 5) + 65536 * static_cast<int>(blockIdx.x);
+        dev_err[2] = pos;
+      }
       return false;
     }
   }
@@ -112,6 +117,20 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
 // Makes generic-proxy shared-memory writes visible to the async proxy (MMA/TMA).
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// 16-byte asynchronous copy global -> shared (L2 only), and the wait for all of the
+// calling thread's outstanding copies. The data lands through the generic proxy: a
+// consumer in the async proxy (tcgen05.mma) needs fence_proxy_async_smem() after the wait.
+__device__ __forceinline__ void cp_async_16(void* dst_smem, const void* src_gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst_smem)), "l"(src_gmem)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// Named barrier over `count` threads (a multiple of 32), id 1..15.
+__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // ---------------------------------------------------------------- TMEM

@@ -5,7 +5,7 @@ Sampling. Workloads 1-6: every chunk and every head (the complete vertical and
 slash index sets of every (chunk, head) pair), and 512 query rows per head,
 uniform without replacement over the sequence from numpy default_rng(seed +
 1000), sorted, the same rows for every head (all 4096 rows at workload 1).
-Workloads 7 and 8 (1M-token variants beyond the five configurations) check a
+Workloads 7, 8 and 9 (1M-token variants beyond the five configurations) check a
 fixed subset of chunks and heads. The oracle side runs in one process per KV
 head group (tests/fullsize_oracle.py), fed chunk by chunk while the GPU loop
 continues.
@@ -36,6 +36,7 @@ PLAN = {
     6: (None, None, 512),
     7: ([0, 15, 31], [0, 21, 39], 64),
     8: ([31], [0, 17], 32),
+    9: ([0, 8, 31], [0, 21, 39], 64),
 }
 
 

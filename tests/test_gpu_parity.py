@@ -437,3 +437,70 @@ def test_empty_and_out_of_range_sizes_are_rejected():
     with pytest.raises(vsb.VsError):  # a chunk of 512 rows, longer than max_chunk = 256
         ctx.sparse_prefill(dev["q"], 0, 512, dev["k"], dev["v"], lists_to_sets([np.arange(4)] * 2, [np.arange(1)] * 2, 8, 8))
     assert ctx.status() == vsb.VS_OK
+
+
+@pytest.mark.parametrize("dca", [None, (2048, 256)])
+def test_sparse_prefill_gathers_scattered_verticals(dca):
+    """A band of slash offsets plus scattered vertical columns (before each chunk and
+    inside it), the shape in which the kernel gathers vertical columns into dense
+    groups instead of executing their key blocks: every row against the oracle, and
+    the executed tiles far below the causal dense count. With DCA (stride 1792) the
+    groups are split at DCA chunk boundaries, each with its own query rotation."""
+    w = small_workload(2, seq_len=6144, chunk=2048, hq=4, hkv=2, n_planted=8)
+    dev, cpu = layer_inputs(w)
+    ctx = make_ctx(w, dca=dca)
+    rng = np.random.default_rng(21)
+    e_all = w.seq_len
+    V = []
+    for h in range(w.hq):
+        cols = rng.choice(e_all, 220, replace=False)
+        cols = np.union1d(cols, np.arange(640, 768))  # one full key block: executed, never gathered
+        V.append(cols.astype(np.int64))
+    S = [np.union1d(np.arange(0, 300), rng.choice(np.arange(300, e_all), 3, replace=False)).astype(np.int64)
+         for _ in range(w.hq)]
+    scale = scale_of(w)
+    dense_tiles = 0
+    executed = 0
+    for cs, e in _chunks(w):
+        sets = lists_to_sets([x[x < e] for x in V], [x[x < e] for x in S], e, e)
+        out = torch.zeros_like(dev["q"])
+        ctx.sparse_prefill(dev["q"], cs, e, dev["k"], dev["v"], sets, out=out, full=True)
+        assert ctx.status() == vsb.VS_OK
+        ex, _ = ctx.prefill_stats()
+        executed += ex
+        dense_tiles += w.hq * sum((r0 // 128 + 1) for r0 in range(cs, e, 128))
+        got = f64(out[:, cs:e])
+        rows = np.arange(cs, e)
+        for h in range(w.hq):
+            vh, sh = V[h][V[h] < e], S[h][S[h] < e]
+            oo, _ = vo.attention_rows(cpu["q"][h, cs:e], rows, cpu["k"][h // w.group], cpu["v"][h // w.group], e,
+                                      vo.membership(e, vh), vo.membership(e, sh), w.rope_base, scale, dca,
+                                      round_out=False)
+            assert_outputs_close(got[h], oo, f"gather dca={dca} cs={cs} h={h}", w=w)
+    assert executed < 0.5 * dense_tiles, (executed, dense_tiles)
+
+
+def test_rewritten_keys_under_a_cached_rotation_are_reported():
+    """The context caches rotated keys per K pointer; keys rewritten in place without
+    vs_context_reset are caught by the sampled re-rotation of a reused cache."""
+    w = small_workload(2, seq_len=1024, chunk=1024, hq=2, hkv=1)
+    dev, _ = layer_inputs(w)
+    for dca in (None, (512, 128)):
+        ctx = make_ctx(w, dca=dca)
+        V, S = [np.arange(0, 1024, 3)] * 2, [np.arange(8)] * 2
+        sets = lists_to_sets(V, S, 1024, 1024)
+        k = dev["k"].clone()
+        ctx.estimate(dev["q"], 0, k, 1024)
+        ctx.sparse_prefill(dev["q"], 0, 1024, k, dev["v"], sets)
+        assert ctx.status() == vsb.VS_OK
+        ctx.estimate(dev["q"], 0, k, 1024)  # reuses both caches: unchanged keys pass
+        ctx.sparse_prefill(dev["q"], 0, 1024, k, dev["v"], sets)
+        assert ctx.status() == vsb.VS_OK
+        k.mul_(2.0)  # another sequence in the same buffer, without a reset
+        ctx.estimate(dev["q"], 0, k, 1024)
+        assert ctx.status() == vsb.VS_ERR_DEVICE_CHECK
+        assert b"keys changed" in ctx.lib.vs_last_error()
+        ctx.reset()
+        ctx.estimate(dev["q"], 0, k, 1024)
+        ctx.sparse_prefill(dev["q"], 0, 1024, k, dev["v"], sets)
+        assert ctx.status() == vsb.VS_OK

@@ -38,6 +38,11 @@ class Workload:
     # s = max(1, seq_len / yarn_train_len), sqrt(1/t) = 0.1 ln(s) + 1 and the logits
     # are divided by t sqrt(D). None: t = 1.
     yarn_train_len: Optional[int] = None
+    # planted retrieval columns: K += planted_k u at the planted positions, Q += planted_q u
+    planted_q: float = 1.5
+    planted_k: float = 4.0
+    # scaled logit added inside the aligned 64 x 64 diagonal blocks (the band clause)
+    band_logit: float = 2.0
 
     @property
     def dca_window(self) -> Optional[int]:
@@ -95,6 +100,14 @@ WORKLOADS: dict[int, Workload] = {
     8: Workload("cfg8_14b_n1m_dca256k_refine_yarn", hq=40, hkv=8, seq_len=1048576, seed=4,
                 n_planted=1024, kv_budget=1000, ks_budget=2048, refine_tau=0.9, dca_chunk=262144,
                 yarn_train_len=262144),
+    # A regime where vertical-slash structure exists: config 5 with the diagonal band at
+    # +15 scaled logits, the planted columns at +10.7 (11 x 11 raw) and the queries' N(0, 1)
+    # part halved. Refinement stops at the base budgets; the selection is the band's
+    # offsets, offset runs that the planted columns induce in the estimation rows, and the
+    # planted columns themselves, scattered over the sequence.
+    9: Workload("cfg9_14b_n1m_dca256k_refine_structured", hq=40, hkv=8, seq_len=1048576, seed=4,
+                n_planted=1024, kv_budget=1000, ks_budget=2048, refine_tau=0.9, dca_chunk=262144,
+                q_scale=0.5, band_logit=15.0, planted_q=11.0, planted_k=11.0),
 }
 
 
@@ -104,7 +117,7 @@ def small_workload(base: int, seq_len: int, chunk: int, *, hq: Optional[int] = N
                    dca_chunk: Optional[int] = None, seed: Optional[int] = None,
                    refine_tau: Optional[float] = -1.0, head_dim: Optional[int] = None,
                    q_scale: Optional[float] = None, yarn_train_len: Optional[int] = None,
-                   name: Optional[str] = None) -> Workload:
+                   name: Optional[str] = None, **extra) -> Workload:
     """A reduced copy of workload `base` (same generator recipe, smaller sizes)."""
     w = WORKLOADS[base]
     kw = dict(seq_len=seq_len, chunk=chunk)
@@ -130,5 +143,6 @@ def small_workload(base: int, seq_len: int, chunk: int, *, hq: Optional[int] = N
         kw["q_scale"] = q_scale
     if yarn_train_len is not None:
         kw["yarn_train_len"] = yarn_train_len
+    kw.update(extra)
     kw["name"] = name or f"{w.name}_small_n{seq_len}_c{chunk}"
     return replace(w, **kw)

@@ -14,12 +14,15 @@ to bf16):
 * Local band ("q_i . k_j += 2 for i - j < 64", in scaled-logit units): for every
   64-aligned block b a random unit vector z_b on the 32 dims of rotary pairs
   32..47 (which turn by at most ~0.02 rad over 64 positions); with
-  a = sqrt(2 sqrt(D)), Q[:, i] += a z_{i // 64} and K[:, j] += a z_{j // 64}, which
-  adds 2 to the scaled logit of every pair inside an aligned 64 x 64 diagonal
-  block.
+  a = sqrt(band_logit sqrt(D)), Q[:, i] += a z_{i // 64} and K[:, j] += a z_{j // 64},
+  which adds band_logit (2) to the scaled logit of every pair inside an aligned
+  64 x 64 diagonal block.
 * V carries no structure.
 * Sparse-regime variant (q_scale != 1): the N(0, 1) part of Q is multiplied by
   q_scale before the structure is added, so base scaled logits have std q_scale.
+* Strengths: the band adds band_logit (default 2) scaled logits; the planted
+  columns use amplitudes planted_q (queries, default 1.5) and planted_k (keys,
+  default 4).
 """
 from __future__ import annotations
 
@@ -72,8 +75,8 @@ def structure(w: Workload) -> dict:
     return {"u": u, "z": z, "planted": planted_positions(w)}
 
 
-def _band_amp(d: int) -> float:
-    return math.sqrt(2.0 * math.sqrt(d))
+def _band_amp(d: int, logit: float = 2.0) -> float:
+    return math.sqrt(logit * math.sqrt(d))
 
 
 def generate_head(w: Workload, tensor: str, head: int, rows: Optional[torch.Tensor] = None,
@@ -92,16 +95,16 @@ def generate_head(w: Workload, tensor: str, head: int, rows: Optional[torch.Tens
     if tensor == "q":
         if w.q_scale != 1.0:
             x *= w.q_scale  # sparse-regime variant: base logits with std q_scale
-        x += 1.5 * st["u"]
-        x += _band_amp(d) * st["z"][pos // 64]
+        x += w.planted_q * st["u"]
+        x += _band_amp(d, w.band_logit) * st["z"][pos // 64]
     elif tensor == "k":
-        x += _band_amp(d) * st["z"][pos // 64]
+        x += _band_amp(d, w.band_logit) * st["z"][pos // 64]
         planted = st["planted"]
         if rows is None:
-            x[planted] += 4.0 * st["u"]
+            x[planted] += w.planted_k * st["u"]
         else:
             hit = torch.isin(pos, planted)
-            x[hit] += 4.0 * st["u"]
+            x[hit] += w.planted_k * st["u"]
     return x.to(torch.bfloat16)
 
 
