@@ -77,6 +77,7 @@ Layout make_layout(const vs_attn_cfg& cfg, int64_t max_seq, int64_t max_chunk) {
   L.sel_part = take(sel_part_bytes(static_cast<int>(hq), kRecallLevels));
   L.hist = take(static_cast<size_t>(L.nsplit_max) * hq * kMaxLevels * sizeof(float));
   L.choice = take(static_cast<size_t>(hq) * 4 * sizeof(int32_t));
+  L.base_rc = take(static_cast<size_t>(hq) * 2 * sizeof(int32_t));
   L.vbits = take(static_cast<size_t>(hq) * L.nwords * sizeof(uint32_t));
   L.sbits = take(static_cast<size_t>(hq) * L.nwords * sizeof(uint32_t));
   L.scum = take(static_cast<size_t>(hq) * (L.nwords + 1) * sizeof(uint32_t));
@@ -374,11 +375,15 @@ extern "C" vs_status vs_refine(vs_ctx* c, const uint16_t* q, int64_t q_rows, int
   VS_TRY(prepare_estimation(c, q, q_rows, q_pos0, k, k_rows, e, st, &nr));
   VS_TRY(launch_select(sel_scratch(c), c->cfg.hq, vert, slash, e_ld, e, kv_budget, ks_budget, nlev, nullptr,
                        v_idx, cap_v, v_cnt, s_off, cap_s, s_cnt, true, false, st));
-  if (c->cfg.refine_dca_positions && c->dca.enabled)
+  const bool dca_recall = c->cfg.refine_dca_positions && c->dca.enabled;
+  if (dca_recall) {
     VS_TRY(run_recall_hist_dca(c, q, q_rows, q_pos0, k, k_rows, e, nr, nlev, st));
-  else
-    VS_TRY(run_recall_hist(c, e, nr, lse, nlev, st));
-  VS_TRY(run_refine_decide(c, e, nr, nlev, tau, kv_budget, ks_budget, recall, st));
+  } else {
+    // heads whose base budgets already reach tau need no histogram of the higher levels
+    VS_TRY(run_recall_base(c, vert, slash, e_ld, e, nr, lse, tau, st));
+    VS_TRY(run_recall_hist(c, e, nr, lse, nlev, st, ws_ptr<int>(c, c->L.base_rc) + c->cfg.hq));
+  }
+  VS_TRY(run_refine_decide(c, e, nr, nlev, tau, kv_budget, ks_budget, recall, !dca_recall, st));
   return launch_select(sel_scratch(c), c->cfg.hq, vert, slash, e_ld, e, kv_budget, ks_budget, nlev,
                        ws_ptr<int32_t>(c, c->L.choice), v_idx, cap_v, v_cnt, s_off, cap_s, s_cnt, false, true,
                        st);

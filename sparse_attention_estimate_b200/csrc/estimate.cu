@@ -54,6 +54,8 @@ struct EstParams {
   float* part_s;      // kSums: [hq][2][2][e_pad + 256]
   const uint8_t* lvl; // kRecall: [hq][2][e_pad]
   float* hist;        // kRecall: [nsplit][hq][kMaxLevels]
+  const int* dec;     // kRecall: heads already decided at the base budgets (nullable); a CTA
+                      // whose g heads all are skips its pass
   int nlev;
   DevCommon dc;
 };
@@ -125,6 +127,11 @@ __global__ void __launch_bounds__(kEstThreads, 1)
                                            ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = blockIdx.y, split = p.split0 + static_cast<int>(blockIdx.x);
+  if (MODE == kRecall && p.dec) {  // uniform over the CTA, before any barrier or allocation
+    bool all = true;
+    for (int hh = 0; hh < p.g; ++hh) all = all && p.dec[G * p.g + hh] != 0;
+    if (all) return;
+  }
   const int b_begin = p.blk0 + static_cast<int>(blockIdx.x) * p.bps;
   const int b_end = min(b_begin + p.bps, p.nblk);
   const int nb = b_end - b_begin;
@@ -487,12 +494,72 @@ __global__ void sums_fixup_kernel(const float* __restrict__ part_v, const float*
   slash[static_cast<int64_t>(h) * e_ld + d] = acc;
 }
 
+// Recall of the base budgets (refinement level 0) per head, from the sums of the
+// estimation pass: the rows' attention mass on the selected elements is the mass of the
+// selected columns (their vertical sums) plus that of the selected offsets (their slash
+// sums) minus the mass of the elements both select, which only these elements' scores
+// give (one dot product each; few at the base budgets). dec[h] = 1 when it reaches tau:
+// the head needs no histogram of the higher levels. One CTA per head.
+__global__ void __launch_bounds__(256) recall_base_kernel(
+    const float* __restrict__ vert, const float* __restrict__ slash, int64_t e_ld, int64_t e, int nr,
+    const uint8_t* __restrict__ lvl, int64_t e_pad, const float* __restrict__ lse,
+    const uint16_t* __restrict__ q_est, int ntile, const uint16_t* __restrict__ k_rot, int64_t k_rows, int g,
+    float scale_log2, float tau, float* __restrict__ rc0, int* __restrict__ dec) {
+  const int h = blockIdx.x, tid = threadIdx.x, hk = h / g, hh = h % g;
+  const uint8_t* lv_v = lvl + static_cast<int64_t>(h) * 2 * e_pad;
+  const uint8_t* lv_s = lv_v + e_pad;
+  const float* vr = vert + static_cast<int64_t>(h) * e_ld;
+  const float* sr = slash + static_cast<int64_t>(h) * e_ld;
+  const int64_t row0 = e - nr;
+  double acc = 0.0;  // vertical + slash - both, over this thread's columns
+  for (int64_t j = tid; j < e; j += blockDim.x) {
+    if (lv_v[j] == 0) acc += vr[j];
+    if (lv_s[j] == 0) acc += sr[j];
+  }
+  for (int64_t j = tid; j < e; j += blockDim.x) {
+    if (lv_v[j] != 0) continue;
+    const uint16_t* kj = k_rot + (static_cast<int64_t>(hk) * k_rows + j) * kD;
+    for (int r = 0; r < nr; ++r) {
+      const int64_t d = row0 + r - j;
+      if (d < 0 || lv_s[d] != 0) continue;
+      const uint16_t* qr = q_est + (static_cast<int64_t>(hk) * ntile * kTile + hh * kEstRows + r) * kD;
+      float dot = 0.f;
+#pragma unroll 8
+      for (int c = 0; c < kD; ++c)
+        dot = fmaf(__uint_as_float(static_cast<uint32_t>(qr[c]) << 16), __uint_as_float(static_cast<uint32_t>(kj[c]) << 16), dot);
+      acc -= exp2f(dot * scale_log2 - lse[static_cast<int64_t>(h) * kEstRows + r] * kLog2e);
+    }
+  }
+  __shared__ double red[256];
+  red[tid] = acc;
+  __syncthreads();
+  for (int o = blockDim.x / 2; o > 0; o >>= 1) {
+    if (tid < o) red[tid] += red[tid + o];
+    __syncthreads();
+  }
+  if (tid == 0) {
+    const float rc = static_cast<float>(red[0] / nr);
+    rc0[h] = rc;
+    dec[h] = rc >= tau ? 1 : 0;
+  }
+}
+
+vs_status run_recall_base(vs_ctx* c, const float* vert, const float* slash, int64_t e_ld, int64_t e, int nr,
+                          const float* lse, float tau, cudaStream_t st) {
+  recall_base_kernel<<<c->cfg.hq, 256, 0, st>>>(
+      vert, slash, e_ld, e, nr, ws_ptr<uint8_t>(c, c->L.lvl), c->L.e_pad, lse,
+      ws_ptr<uint16_t>(c, c->L.q_est), c->L.ntile, ws_ptr<uint16_t>(c, c->L.k_cont), c->max_seq,
+      c->cfg.hq / c->cfg.hkv, c->cfg.softmax_scale * kLog2e, tau, ws_ptr<float>(c, c->L.base_rc),
+      ws_ptr<int>(c, c->L.base_rc) + c->cfg.hq);
+  return launched("recall_base_kernel launch");
+}
+
 // One estimation-kernel launch over key blocks [blk0, blk1) with the rotated rows
 // in q_buf and the rotated keys in k_buf; its splits write partial outputs from
 // index split0 on. *nsplit_out gets the number of splits used.
 static vs_status launch_est_range(vs_ctx* c, int mode, int64_t e, int nr, const float* lse, int nlev,
                                   int blk0, int blk1, int split0, int max_splits, size_t q_buf,
-                                  size_t k_buf, int* nsplit_out, cudaStream_t st) {
+                                  size_t k_buf, int* nsplit_out, cudaStream_t st, const int* dec = nullptr) {
   const int hkv = c->cfg.hkv, g = c->cfg.hq / c->cfg.hkv;
   const int nblk = blk1 - blk0;
   if (nblk <= 0) {
@@ -530,6 +597,7 @@ static vs_status launch_est_range(vs_ctx* c, int mode, int64_t e, int nr, const 
   p.part_s = ws_ptr<float>(c, c->L.part_s);
   p.lvl = ws_ptr<uint8_t>(c, c->L.lvl);
   p.hist = ws_ptr<float>(c, c->L.hist);
+  p.dec = dec;
   p.nlev = nlev;
   p.dc = dev_common(c);
   const size_t smem = sizeof(EstSmem) + 1024;
@@ -550,9 +618,9 @@ static vs_status launch_est_range(vs_ctx* c, int mode, int64_t e, int nr, const 
 // All key blocks of [0, e) with continuous positions (estimation rows in q_est,
 // keys in the continuous rotated cache).
 static vs_status launch_est(vs_ctx* c, int mode, int64_t e, int nr, const float* lse, int nlev,
-                            int* nsplit_out, cudaStream_t st) {
+                            int* nsplit_out, cudaStream_t st, const int* dec = nullptr) {
   return launch_est_range(c, mode, e, nr, lse, nlev, 0, static_cast<int>(ceil_div(e, kTile)), 0,
-                          c->L.nsplit_max, c->L.q_est, c->L.k_cont, nsplit_out, st);
+                          c->L.nsplit_max, c->L.q_est, c->L.k_cont, nsplit_out, st, dec);
 }
 
 vs_status run_estimate(vs_ctx* c, const uint16_t* q, int64_t q_rows, int64_t q_pos0,
@@ -637,9 +705,9 @@ vs_status run_recall_hist_dca(vs_ctx* c, const uint16_t* q, int64_t q_rows, int6
 }
 
 vs_status run_recall_hist(vs_ctx* c, int64_t e, int nr, const float* lse, int nlev,
-                          cudaStream_t st) {
+                          cudaStream_t st, const int* dec) {
   int nsplit = 0;
-  vs_status s = launch_est(c, kRecall, e, nr, lse, nlev, &nsplit, st);
+  vs_status s = launch_est(c, kRecall, e, nr, lse, nlev, &nsplit, st, dec);
   c->hist_nsplit = nsplit;
   return s;
 }

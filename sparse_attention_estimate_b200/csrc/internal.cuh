@@ -61,6 +61,7 @@ struct Layout {
   size_t sel_state, sel_part; // radix-select state and per-segment histograms
   size_t hist;                // recall histograms [nsplit_max][hq][kMaxLevels]
   size_t choice;              // chosen level per head [hq] + flags
+  size_t base_rc;             // recall at the base budgets [hq] fp32, then decided flags [hq] int
   size_t vbits, sbits, scum;  // bitmaps [hq][nwords] and slash prefix counts
   size_t gbits, gcum;         // gathered vertical columns [hq][nwords] and their prefix counts
   size_t gscan;               // gathered columns before each key block [hq][nblk + 1]
@@ -154,7 +155,9 @@ vs_status run_recall_hist_dca(vs_ctx* c, const uint16_t* q, int64_t q_rows, int6
                               const uint16_t* k, int64_t k_rows, int64_t e, int nr, int nlev,
                               cudaStream_t st);
 vs_status run_recall_hist(vs_ctx* c, int64_t e, int nr, const float* lse, int nlev,
-                          cudaStream_t st);
+                          cudaStream_t st, const int* dec = nullptr);
+vs_status run_recall_base(vs_ctx* c, const float* vert, const float* slash, int64_t e_ld, int64_t e, int nr,
+                          const float* lse, float tau, cudaStream_t st);
 // select.cu
 constexpr int kSelMaxSegments = 64;  // segments (CTAs) per (head, array), at most
 // Scratch of the selection kernels (the context's workspace, or the no-alloc array).
@@ -175,7 +178,7 @@ vs_status launch_select(const SelScratch& sc, int hq, const float* vert, const f
                         int32_t* v_idx, int32_t cap_v, int32_t* v_cnt, int32_t* s_off, int32_t cap_s,
                         int32_t* s_cnt, bool thresholds_and_levels, bool compact, cudaStream_t st);
 vs_status run_refine_decide(vs_ctx* c, int64_t e, int nr, int nlev, float tau, int32_t* kv,
-                            int32_t* ks, float* recall, cudaStream_t st);
+                            int32_t* ks, float* recall, bool base_decided, cudaStream_t st);
 vs_status run_budgets_max(int hq, const int32_t* kv, const int32_t* ks, int32_t* kv_acc, int32_t* ks_acc,
                           cudaStream_t st);
 // attn.cu

@@ -432,10 +432,18 @@ __global__ void __launch_bounds__(kSelThreads) compact_write_kernel(
 
 __global__ void refine_decide_kernel(const float* __restrict__ hist, int nsplit, int hq, int nlev,
                                      int nr, int64_t e, float tau, int32_t* kv, int32_t* ks,
-                                     float* recall, int32_t* choice) {
+                                     float* recall, int32_t* choice, const float* __restrict__ base_rc,
+                                     const int* __restrict__ base_dec) {
   const int h = blockIdx.x * blockDim.x + threadIdx.x;
   if (h >= hq) return;
   int64_t kv0 = kv[h] < 0 ? 0 : kv[h], ks0 = ks[h] < 0 ? 0 : ks[h];
+  if (base_dec && base_dec[h]) {  // the base budgets reach tau (their recall from the sums)
+    choice[h] = 0;
+    kv[h] = static_cast<int32_t>(kv0 > e ? e : kv0);
+    ks[h] = static_cast<int32_t>(ks0 > e ? e : ks0);
+    recall[h] = base_rc[h];
+    return;
+  }
   double cum = 0.0;
   int chosen = nlev - 1;
   int64_t kvt = 0, kst = 0;
@@ -477,10 +485,11 @@ vs_status run_budgets_max(int hq, const int32_t* kv, const int32_t* ks, int32_t*
 }
 
 vs_status run_refine_decide(vs_ctx* c, int64_t e, int nr, int nlev, float tau, int32_t* kv,
-                            int32_t* ks, float* recall, cudaStream_t st) {
+                            int32_t* ks, float* recall, bool base_decided, cudaStream_t st) {
   refine_decide_kernel<<<static_cast<unsigned>(ceil_div(c->cfg.hq, 64)), 64, 0, st>>>(
       ws_ptr<float>(c, c->L.hist), c->hist_nsplit, c->cfg.hq, nlev, nr, e, tau, kv, ks, recall,
-      ws_ptr<int32_t>(c, c->L.choice));
+      ws_ptr<int32_t>(c, c->L.choice), base_decided ? ws_ptr<float>(c, c->L.base_rc) : nullptr,
+      base_decided ? ws_ptr<int>(c, c->L.base_rc) + c->cfg.hq : nullptr);
   return launched("refine_decide_kernel launch");
 }
 
