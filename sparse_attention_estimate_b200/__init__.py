@@ -32,7 +32,7 @@ EXPORTS = ("vs_workspace_size", "vs_context_create", "vs_context_destroy", "vs_c
            "vs_set_wait_limit", "dca_remap", "vs_estimate", "vs_select", "vs_refine",
            "vs_sparse_prefill", "vs_prefill_stats", "vs_status_poll", "vs_selftest_wait_timeout",
            "vs_last_error", "vs_set_prefill_events", "vs_kernel_launches", "vs_select_noalloc",
-           "vs_calibrate_accumulate")
+           "vs_calibrate_accumulate", "vs_set_deterministic")
 
 
 class VsError(RuntimeError):
@@ -67,6 +67,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "vs_context_destroy": [P],
         "vs_context_reset": [P],
         "vs_set_wait_limit": [P, U64],
+        "vs_set_deterministic": [P, I32],
         "dca_remap": [P, I64, I64, P, P, P, P, P],
         "vs_estimate": [P, P, I64, I64, P, I64, I64, P, P, I64, P, P],
         "vs_select": [P, P, P, I64, I64, P, P, P, I32, P, P, I32, P, P],
@@ -198,6 +199,10 @@ class Context:
 
     def set_wait_limit(self, ns: int):
         _check(self.lib.vs_set_wait_limit(self.handle, ns))
+
+    def set_deterministic(self, on: bool):
+        """Bitwise reproducible prefill (every work list swept from its start)."""
+        _check(self.lib.vs_set_deterministic(self.handle, 1 if on else 0))
 
     def status(self) -> int:
         """Synchronises and returns (and clears) the device error word status."""

@@ -78,6 +78,7 @@ Layout make_layout(const vs_attn_cfg& cfg, int64_t max_seq, int64_t max_chunk) {
   L.hist = take(static_cast<size_t>(L.nsplit_max) * hq * kMaxLevels * sizeof(float));
   L.choice = take(static_cast<size_t>(hq) * 4 * sizeof(int32_t));
   L.base_rc = take(static_cast<size_t>(hq) * 2 * sizeof(int32_t));
+  L.base_part = take(static_cast<size_t>(hq) * kBaseSplits * sizeof(double));
   L.vbits = take(static_cast<size_t>(hq) * L.nwords * sizeof(uint32_t));
   L.sbits = take(static_cast<size_t>(hq) * L.nwords * sizeof(uint32_t));
   L.scum = take(static_cast<size_t>(hq) * (L.nwords + 1) * sizeof(uint32_t));
@@ -87,8 +88,9 @@ Layout make_layout(const vs_attn_cfg& cfg, int64_t max_seq, int64_t max_chunk) {
   L.glist = take(static_cast<size_t>(hq) * L.e_pad * sizeof(int32_t));
   L.gtab = take(static_cast<size_t>(hq) * L.gcap * 4 * sizeof(int32_t));
   L.gkoff = take(static_cast<size_t>(hq) * (L.nkmax + 1) * sizeof(int32_t));
-  L.sched = take(static_cast<size_t>(hq) * L.npairs * L.nsched * sizeof(int32_t));
+  L.sched = take(static_cast<size_t>(hq) * L.npairs * 2 * L.nsched * sizeof(int32_t));
   L.sched_cnt = take(static_cast<size_t>(hq) * L.npairs * sizeof(int32_t));
+  L.sweep = take(static_cast<size_t>(hq) * sizeof(int32_t));
   L.total = off;
   return L;
 }
@@ -224,6 +226,7 @@ extern "C" vs_status vs_context_create(const vs_attn_cfg* cfg, int64_t max_seq, 
   c->device = dev;
   c->num_sms = sms;
   c->wait_ns = 2000000000ull;
+  c->deterministic = false;
   c->dca.enabled = cfg->dca_enabled ? 1 : 0;
   c->dca.C = cfg->dca_chunk_size;
   c->dca.W = cfg->dca_local_window;
@@ -267,6 +270,12 @@ extern "C" vs_status vs_set_wait_limit(vs_ctx* c, uint64_t ns) {
   VS_REQUIRE(c, VS_ERR_INVALID_ARG, "context is NULL");
   VS_REQUIRE(ns >= 1000, VS_ERR_INVALID_ARG, "wait limit below 1 us");
   c->wait_ns = ns;
+  return VS_OK;
+}
+
+extern "C" vs_status vs_set_deterministic(vs_ctx* c, int on) {
+  VS_REQUIRE(c, VS_ERR_INVALID_ARG, "context is NULL");
+  c->deterministic = on != 0;
   return VS_OK;
 }
 

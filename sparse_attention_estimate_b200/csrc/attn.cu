@@ -37,6 +37,9 @@
 namespace vs {
 
 constexpr int kAttnThreads = 384;
+// Work lists of at least this many entries (K and V of 1024 key blocks per KV head: 64 MB)
+// are swept from where the other CTAs of their head are loading (see attn_kernel).
+constexpr int kSweepMin = 1024;
 // Register budgets after the role split: warpgroup 0 (TMA producer, MMA issuer, two
 // idle warps) keeps 112 per thread, the two softmax warpgroups take 192 each:
 // 128 x 112 + 256 x 192 = 63488 <= 384 x 168 (the launch's 64512).
@@ -317,7 +320,7 @@ __global__ void __launch_bounds__(256) schedule_kernel(
   const int64_t sblk = dca.enabled ? dca.S / kTile : nb;
   const int64_t nk = (nb + sblk - 1) / sblk;
   const int64_t nk_all = ((e + kTile - 1) / kTile + sblk - 1) / sblk;  // key chunks of the plan
-  int32_t* out = sched + (static_cast<int64_t>(h) * npairs_ws + pair) * nsched;
+  int32_t* out = sched + (static_cast<int64_t>(h) * npairs_ws + pair) * 2 * nsched;
   auto gl_last = [&](int hh, const int4& d) {  // last column of a group
     return static_cast<int64_t>(glist[static_cast<int64_t>(hh) * e_pad + d.x + d.y - 1]);
   };
@@ -376,6 +379,12 @@ __global__ void __launch_bounds__(256) schedule_kernel(
       emit(flags != 0, static_cast<int32_t>(b) | (flags << 24) | (hg0 ? kEntFlag : 0));
     }
   }
+  // A list long enough to be swept from another start is written twice in a row, so that
+  // the attention CTA reads entries start .. start + n - 1 with no wrap-around.
+  if (running >= kSweepMin) {
+    __syncthreads();
+    for (int i = tid; i < running; i += blockDim.x) out[running + i] = out[i];
+  }
   if (tid == 0) {
     // the list's length, and bit 30 when it holds gather groups
     sched_cnt[static_cast<int64_t>(h) * npairs_ws + pair] = running | (groups > 0 ? kCntGroups : 0);
@@ -404,6 +413,8 @@ struct AttnParams {
   const int4* gtab;
   int64_t e_pad, gcap;
   int dca_sblk;  // key blocks per DCA chunk (S / 128), 0 without DCA
+  int* sweep;    // per query head: list position last loaded by one of its CTAs (a hint)
+  int rotate;    // lists of kSweepMin entries or more start at that position
   // row sources of the gathered groups: rotated keys and values, [hkv][rows][128]
   const uint16_t* k_rot;
   int64_t k_rows;
@@ -426,6 +437,7 @@ struct __align__(1024) AttnSmem {
   uint32_t tmem_base;
   int abort_word;
   int gather_ok;  // a stage wait's outcome, shared among the gather threads
+  int start;      // first list entry of this CTA's sweep
 };
 
 __device__ __forceinline__ float ex2a(float x) {
@@ -474,7 +486,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int pair = p.npairs - 1 - rg / p.g;
   const int h = hk * p.g + rg % p.g;
   const int64_t R0 = p.q_pos0 + static_cast<int64_t>(pair) * 256;  // tile 0's first row
-  const int32_t* list = p.sched + (static_cast<int64_t>(h) * p.npairs_ws + pair) * p.nsched;
+  const int32_t* list = p.sched + (static_cast<int64_t>(h) * p.npairs_ws + pair) * 2 * p.nsched;
   // DCA chunks of the two query tiles (fixed for the CTA)
   const int qc0 = p.dca.enabled ? static_cast<int>(R0 / p.dca.S) : 0;
   const int qc1 = p.dca.enabled ? static_cast<int>((R0 + kTile) / p.dca.S) : 0;
@@ -497,6 +509,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     mbar_init(&s.o_final, 1);
     mbar_init(&s.drain, 1);
     s.abort_word = 0;
+    // Sweep start: where a CTA of the same query head loaded last. Once a KV head's keys
+    // and values outgrow L2, CTAs that all sweep from block 0 drift apart (SMs run at
+    // slightly different speeds, and each takes the next CTA when its own ends) until the
+    // blocks a CTA reads have left L2 before the next one reaches them. Joining the CTAs
+    // in flight keeps them within a few hundred blocks of each other. The position is kept
+    // per query head, not per KV head: heads whose masks cost different time per block
+    // then form one group each instead of one spread-out group. A list of n entries is
+    // stored twice in a row, so the sweep start .. start + n - 1 needs no wrap-around;
+    // the order of the entries changes only the summation order of the online softmax.
+    int start = 0;
+    if (p.rotate && n >= kSweepMin)
+      start = static_cast<int>(static_cast<uint32_t>(__ldcg(p.sweep + h)) % static_cast<uint32_t>(n));
+    s.start = start;
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -514,12 +539,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (warp == 0) {
       // ------------------------------------------------------------ TMA producer
       if (lane == 0 && n > 0) {
+        const int start = s.start;
+        const int32_t* lst = list + start;
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
         int cls[2];
         int qchg[2] = {0, 0};
-        const int kc0 = entry_kchunk(list[0], p.gtab, p.gcap, h, p.dca_sblk);
+        const int kc0 = entry_kchunk(lst[0], p.gtab, p.gcap, h, p.dca_sblk);
         for (int t = 0; t < 2; ++t) {
           cls[t] = dca_class(t ? qc1 : qc0, kc0);
           mbar_arrive_expect_tx(&s.q_full[t], 2 * kTileBytes);
@@ -533,12 +560,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // draining the copies in flight when the CTA aborts
         int nst[2] = {0, 0}, kph[2] = {-1, -1}, vph[2] = {-1, -1};
         bool ok = true;
-        int32_t ent = list[0];  // schedule entries are read one block ahead of use
+        int32_t ent = lst[0];  // schedule entries are read one block ahead of use
         for (int j = 0; j < n && ok; ++j) {
           const int32_t cur = ent;
           const int b = cur & 0xFFFFFF;
           const bool grp = (cur & kEntGroup) != 0;  // a gather group: warps 2-3 load its K and V
-          ent = j + 1 < n ? ld_keep_s32(list + j + 1) : 0;
+          ent = j + 1 < n ? ld_keep_s32(lst + j + 1) : 0;
           const int st = j & 1;
           // K(j) first: the MMA warp releases a Q tile only after issuing S0(j).
           // Both loaders (this one and the gather warps) wait for every entry's stage to
@@ -551,6 +578,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             tma_load_3d(s.k[st][0], &tmK, &s.k_full[st], 0, b * kTile, hk);
             tma_load_3d(s.k[st][1], &tmK, &s.k_full[st], 64, b * kTile, hk);
             kph[st] = nst[st];
+          }
+          if (p.rotate && n >= kSweepMin && (j & 63) == 0) {  // where this CTA is now
+            const int pos = start + j;
+            __stcg(p.sweep + h, pos >= n ? pos - n : pos);
           }
           if (j > 0) {
             const int kc = entry_kchunk(cur, p.gtab, p.gcap, h, p.dca_sblk);
@@ -600,10 +631,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const uint32_t tS[2] = {tbase, tbase + 128};
           const uint32_t tO[2] = {tbase + 256, tbase + 384};
           int cls[2], qph[2] = {1, 1};
-          const int kc0 = entry_kchunk(list[0], p.gtab, p.gcap, h, p.dca_sblk);
+          const int32_t* lst = list + s.start;
+          const int kc0 = entry_kchunk(lst[0], p.gtab, p.gcap, h, p.dca_sblk);
           cls[0] = dca_class(qc0, kc0);
           cls[1] = dca_class(qc1, kc0);
-          int32_t ent1 = n > 1 ? list[1] : 0;  // entry of block j + 1, read a block ahead
+          int32_t ent1 = n > 1 ? lst[1] : 0;  // entry of block j + 1, read a block ahead
           // descriptor words of the operand tiles (K-major Q and K, MN-major V; 128-byte swizzle)
           const uint32_t dhi = smem_desc_sw128_hi(1024);
           const uint32_t qlo[2] = {smem_desc_sw128_lo(smem_u32(&s.q[0][0][0]), 16),
@@ -642,7 +674,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const bool more = j + 1 < n;
             const int st1 = (j + 1) & 1;
             const int kc1 = more ? entry_kchunk(ent1, p.gtab, p.gcap, h, p.dca_sblk) : 0;
-            ent1 = j + 2 < n ? ld_keep_s32(list + j + 2) : 0;
+            ent1 = j + 2 < n ? ld_keep_s32(lst + j + 2) : 0;
             const int c0 = more ? dca_class(qc0, kc1) : cls[0];
             const int c1 = more ? dca_class(qc1, kc1) : cls[1];
             // V(j) and K(j+1) normally landed long ago: wait for them before P_0(j), so
@@ -700,14 +732,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // column; their scores are masked). Thread g copies tile rows g and g + 64.
       const int gtid = tid - 64;
       const int32_t* gl = p.glist + static_cast<int64_t>(h) * p.e_pad;
-      int32_t ent = n > 0 ? list[0] : 0;
+      const int32_t* lst = list + s.start;
+      int32_t ent = n > 0 ? lst[0] : 0;
       bool ok = has_groups;  // lists without groups are the TMA producer's alone
       // Every entry's stage-empty phases are waited for (by thread 0, the outcome shared
       // through the named barrier), as in the TMA producer: a parity wait is exact only
       // for the phase right after the last one waited for.
       for (int j = 0; j < n && ok; ++j) {
         const int32_t cur = ent;
-        ent = j + 1 < n ? ld_keep_s32(list + j + 1) : 0;
+        ent = j + 1 < n ? ld_keep_s32(lst + j + 1) : 0;
         const bool grp = (cur & kEntGroup) != 0;
         const int st = j & 1;
         int64_t col[2] = {0, 0};
@@ -761,12 +794,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t* vb = p.vbits + static_cast<int64_t>(h) * p.nwords;
     const uint32_t* sb = p.sbits + static_cast<int64_t>(h) * p.nwords;
     float m_run = -INFINITY, l_run = 0.f;
-    int32_t ent = n > 0 ? list[0] : 0;  // schedule entry of block j, read a block ahead
+    const int32_t* lst = list + s.start;
+    int32_t ent = n > 0 ? lst[0] : 0;  // schedule entry of block j, read a block ahead
     unsigned long long useful = 0;
     bool ok = true;
     for (int j = 0; j < n && ok; ++j) {
       const int32_t entry = ent;
-      ent = j + 1 < n ? ld_keep_s32(list + j + 1) : 0;
+      ent = j + 1 < n ? ld_keep_s32(lst + j + 1) : 0;
       const int64_t k0 = static_cast<int64_t>(entry & 0xFFFFFF) * kTile;
       const int state = (entry >> (24 + 2 * t)) & 3;
       // element mask of this row over the block's (or gather group's) 128 keys
@@ -1048,6 +1082,8 @@ vs_status run_sparse_prefill(vs_ctx* c, const uint16_t* q, int64_t q_rows, int64
   ap.sched = ws_ptr<int32_t>(c, L.sched);
   ap.sched_cnt = ws_ptr<int32_t>(c, L.sched_cnt);
   ap.npairs_ws = static_cast<int>(L.npairs);
+  ap.sweep = ws_ptr<int>(c, L.sweep);
+  ap.rotate = c->deterministic ? 0 : 1;
   ap.nsched = L.nsched;
   ap.vbits = vbits;
   ap.sbits = sbits;

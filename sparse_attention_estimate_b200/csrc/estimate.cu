@@ -498,60 +498,125 @@ __global__ void sums_fixup_kernel(const float* __restrict__ part_v, const float*
 // estimation pass: the rows' attention mass on the selected elements is the mass of the
 // selected columns (their vertical sums) plus that of the selected offsets (their slash
 // sums) minus the mass of the elements both select, which only these elements' scores
-// give (one dot product each; few at the base budgets). dec[h] = 1 when it reaches tau:
-// the head needs no histogram of the higher levels. One CTA per head.
+// give (one dot product each; few at the base budgets, most of them near the diagonal).
+// A grid of (kBaseSplits, hq) CTAs takes one slice of the columns each, 4096 at a time:
+// every thread scans 16 columns' level bytes at once, adds the selected sums and queues
+// its selected vertical columns in shared memory; then each warp takes queued columns in
+// turn, its lanes the estimation rows (r and r + 32), and subtracts exp(s - lse) of the
+// rows whose offset is selected too. The CTAs' sums are added in a fixed order by
+// recall_base_finish_kernel (the result does not depend on scheduling), which sets
+// dec[h] = 1 when the recall reaches tau: the head then needs no histogram of the
+// higher levels.
+constexpr int kBaseRound = 4096;  // columns per round of the base-recall scan
 __global__ void __launch_bounds__(256) recall_base_kernel(
     const float* __restrict__ vert, const float* __restrict__ slash, int64_t e_ld, int64_t e, int nr,
     const uint8_t* __restrict__ lvl, int64_t e_pad, const float* __restrict__ lse,
     const uint16_t* __restrict__ q_est, int ntile, const uint16_t* __restrict__ k_rot, int64_t k_rows, int g,
-    float scale_log2, float tau, float* __restrict__ rc0, int* __restrict__ dec) {
-  const int h = blockIdx.x, tid = threadIdx.x, hk = h / g, hh = h % g;
-  const uint8_t* lv_v = lvl + static_cast<int64_t>(h) * 2 * e_pad;
+    float scale_log2, double* __restrict__ part) {
+  __shared__ int32_t queue[kBaseRound];
+  __shared__ int nq;
+  __shared__ double red[256];
+  const int h = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int hk = h / g, hh = h % g;
+  const uint8_t* lv_v = lvl + static_cast<int64_t>(h) * 2 * e_pad;  // 16-byte aligned rows
   const uint8_t* lv_s = lv_v + e_pad;
   const float* vr = vert + static_cast<int64_t>(h) * e_ld;
   const float* sr = slash + static_cast<int64_t>(h) * e_ld;
   const int64_t row0 = e - nr;
-  double acc = 0.0;  // vertical + slash - both, over this thread's columns
-  for (int64_t j = tid; j < e; j += blockDim.x) {
-    if (lv_v[j] == 0) acc += vr[j];
-    if (lv_s[j] == 0) acc += sr[j];
+  const int64_t per = ((e + 15) / 16 + gridDim.x - 1) / gridDim.x * 16;  // columns per CTA
+  const int64_t j0 = static_cast<int64_t>(blockIdx.x) * per;
+  const int64_t j1 = j0 + per < e ? j0 + per : e;
+  // this lane's estimation rows, their lse (log2 units) and query rows (256-byte aligned)
+  const uint16_t* qbase = q_est + (static_cast<int64_t>(hk) * ntile * kTile + hh * kEstRows) * kD;
+  float lse2[2];
+  for (int t = 0; t < 2; ++t) {
+    const int r = lane + 32 * t;
+    lse2[t] = r < nr ? lse[static_cast<int64_t>(h) * kEstRows + r] * kLog2e : 0.f;
   }
-  for (int64_t j = tid; j < e; j += blockDim.x) {
-    if (lv_v[j] != 0) continue;
-    const uint16_t* kj = k_rot + (static_cast<int64_t>(hk) * k_rows + j) * kD;
-    for (int r = 0; r < nr; ++r) {
-      const int64_t d = row0 + r - j;
-      if (d < 0 || lv_s[d] != 0) continue;
-      const uint16_t* qr = q_est + (static_cast<int64_t>(hk) * ntile * kTile + hh * kEstRows + r) * kD;
-      float dot = 0.f;
-#pragma unroll 8
-      for (int c = 0; c < kD; ++c)
-        dot = fmaf(__uint_as_float(static_cast<uint32_t>(qr[c]) << 16), __uint_as_float(static_cast<uint32_t>(kj[c]) << 16), dot);
-      acc -= exp2f(dot * scale_log2 - lse[static_cast<int64_t>(h) * kEstRows + r] * kLog2e);
+  double acc = 0.0;  // vertical + slash - both
+  for (int64_t rb = j0; rb < j1; rb += kBaseRound) {
+    if (tid == 0) nq = 0;
+    __syncthreads();
+    const int64_t jb = rb + 16 * tid;
+    if (jb < j1) {
+      const uint4 wv = *reinterpret_cast<const uint4*>(lv_v + jb);
+      const uint4 ws = *reinterpret_cast<const uint4*>(lv_s + jb);
+      const uint32_t av[4] = {wv.x, wv.y, wv.z, wv.w}, as[4] = {ws.x, ws.y, ws.z, ws.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        // a zero byte is an element of the base level; most words hold none
+        const uint32_t zv = __vcmpeq4(av[q], 0u), zs = __vcmpeq4(as[q], 0u);
+        if ((zv | zs) == 0u) continue;
+        for (int b = 0; b < 4; ++b) {
+          const int64_t j = jb + 4 * q + b;
+          if (j >= j1) break;
+          if ((zs >> (8 * b)) & 1u) acc += sr[j];
+          if ((zv >> (8 * b)) & 1u) {
+            acc += vr[j];
+            queue[atomicAdd(&nq, 1)] = static_cast<int32_t>(j - rb);
+          }
+        }
+      }
     }
+    __syncthreads();
+    const int n = nq;
+    for (int i = warp; i < n; i += 8) {
+      const int64_t j = rb + queue[i];
+      const uint4* kj = reinterpret_cast<const uint4*>(k_rot + (static_cast<int64_t>(hk) * k_rows + j) * kD);
+      for (int t = 0; t < 2; ++t) {
+        const int r = lane + 32 * t;
+        const int64_t d = row0 + r - j;  // this element's offset
+        if (r >= nr || d < 0 || lv_s[d] != 0) continue;
+        const uint4* qr = reinterpret_cast<const uint4*>(qbase + static_cast<int64_t>(r) * kD);
+        float dot = 0.f;
+#pragma unroll 4
+        for (int c = 0; c < kD / 8; ++c) {
+          const uint4 a = qr[c], b = kj[c];
+          const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            dot = fmaf(__uint_as_float(aw[u] << 16), __uint_as_float(bw[u] << 16), dot);
+            dot = fmaf(__uint_as_float(aw[u] & 0xFFFF0000u), __uint_as_float(bw[u] & 0xFFFF0000u), dot);
+          }
+        }
+        acc -= exp2f(dot * scale_log2 - lse2[t]);
+      }
+    }
+    __syncthreads();  // the queue is refilled next round
   }
-  __shared__ double red[256];
   red[tid] = acc;
   __syncthreads();
   for (int o = blockDim.x / 2; o > 0; o >>= 1) {
     if (tid < o) red[tid] += red[tid + o];
     __syncthreads();
   }
-  if (tid == 0) {
-    const float rc = static_cast<float>(red[0] / nr);
-    rc0[h] = rc;
-    dec[h] = rc >= tau ? 1 : 0;
-  }
+  if (tid == 0) part[static_cast<int64_t>(h) * gridDim.x + blockIdx.x] = red[0];
+}
+
+__global__ void recall_base_finish_kernel(const double* __restrict__ part, int nsplit, int hq, int nr,
+                                          float tau, float* __restrict__ rc0, int* __restrict__ dec) {
+  const int h = blockIdx.x * blockDim.x + threadIdx.x;
+  if (h >= hq) return;
+  double sum = 0.0;
+  for (int i = 0; i < nsplit; ++i) sum += part[static_cast<int64_t>(h) * nsplit + i];
+  const float rc = static_cast<float>(sum / nr);
+  rc0[h] = rc;
+  dec[h] = rc >= tau ? 1 : 0;
 }
 
 vs_status run_recall_base(vs_ctx* c, const float* vert, const float* slash, int64_t e_ld, int64_t e, int nr,
                           const float* lse, float tau, cudaStream_t st) {
-  recall_base_kernel<<<c->cfg.hq, 256, 0, st>>>(
+  const int hq = c->cfg.hq;
+  double* part = ws_ptr<double>(c, c->L.base_part);
+  recall_base_kernel<<<dim3(kBaseSplits, hq), 256, 0, st>>>(
       vert, slash, e_ld, e, nr, ws_ptr<uint8_t>(c, c->L.lvl), c->L.e_pad, lse,
       ws_ptr<uint16_t>(c, c->L.q_est), c->L.ntile, ws_ptr<uint16_t>(c, c->L.k_cont), c->max_seq,
-      c->cfg.hq / c->cfg.hkv, c->cfg.softmax_scale * kLog2e, tau, ws_ptr<float>(c, c->L.base_rc),
-      ws_ptr<int>(c, c->L.base_rc) + c->cfg.hq);
-  return launched("recall_base_kernel launch");
+      hq / c->cfg.hkv, c->cfg.softmax_scale * kLog2e, part);
+  vs_status s = launched("recall_base_kernel launch");
+  if (s != VS_OK) return s;
+  recall_base_finish_kernel<<<(hq + 127) / 128, 128, 0, st>>>(
+      part, kBaseSplits, hq, nr, tau, ws_ptr<float>(c, c->L.base_rc), ws_ptr<int>(c, c->L.base_rc) + hq);
+  return launched("recall_base_finish_kernel launch");
 }
 
 // One estimation-kernel launch over key blocks [blk0, blk1) with the rotated rows

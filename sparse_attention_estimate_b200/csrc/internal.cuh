@@ -20,6 +20,7 @@ constexpr int kMaxG = 8;         // largest GQA group the estimation kernel tile
 constexpr int kMaxLevels = 32;   // selection levels stored per (head, array)
 constexpr int kRecallLevels = 20;  // refinement levels (max_iters <= 19)
 constexpr int kSPad = 4;         // zero words in front of each slash bitmap
+constexpr int kBaseSplits = 32;  // CTAs per head of the base-recall scan
 constexpr int kEstRows = 64;     // estimation rows per head (upper bound of last_q)
 
 // Parameters every kernel with a bounded wait receives.
@@ -62,13 +63,16 @@ struct Layout {
   size_t hist;                // recall histograms [nsplit_max][hq][kMaxLevels]
   size_t choice;              // chosen level per head [hq] + flags
   size_t base_rc;             // recall at the base budgets [hq] fp32, then decided flags [hq] int
+  size_t base_part;           // partial sums of the base-recall scan [hq][kBaseSplits] fp64
   size_t vbits, sbits, scum;  // bitmaps [hq][nwords] and slash prefix counts
   size_t gbits, gcum;         // gathered vertical columns [hq][nwords] and their prefix counts
   size_t gscan;               // gathered columns before each key block [hq][nblk + 1]
   size_t glist;               // gathered columns, ascending [hq][e_pad]
   size_t gtab;                // gather groups [hq][gcap] (start, count, DCA key chunk, first column)
   size_t gkoff;               // first group of each DCA key chunk [hq][nkmax + 1]
-  size_t sched, sched_cnt;    // work lists [hq][npairs][nsched] and counts [hq][npairs]
+  size_t sched, sched_cnt;    // work lists [hq][npairs][2 * nsched] (each list written twice in a row)
+                              // and their lengths [hq][npairs]
+  size_t sweep;               // list position of each query head's attention CTAs [hq] (a hint)
   size_t total;
   int64_t rows_pad;           // max_chunk rounded up to 256
   int64_t e_pad;              // max_seq rounded up to 128
@@ -98,6 +102,7 @@ struct vs_ctx {
   vs::Layout L;
   int device, num_sms;
   uint64_t wait_ns;
+  bool deterministic;  // attention CTAs sweep their lists from the start
   vs::DcaParams dca;
   vs::KCache kc, kd;  // continuous / DCA rotated key caches
   int hist_nsplit;    // splits of the last recall-histogram launch

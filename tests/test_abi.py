@@ -79,6 +79,7 @@ def test_calls_reject_null_context(lib):
                                  None) == vsb.VS_ERR_INVALID_ARG
     assert lib.vs_context_reset(None) == vsb.VS_ERR_INVALID_ARG
     assert lib.vs_set_wait_limit(None, 10 ** 9) == vsb.VS_ERR_INVALID_ARG
+    assert lib.vs_set_deterministic(None, 1) == vsb.VS_ERR_INVALID_ARG
 
 
 @pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="checks the behaviour without a CUDA device")

@@ -310,6 +310,36 @@ def test_sparse_prefill_is_deterministic(case):
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
 
 
+def test_long_lists_swept_from_a_shared_start():
+    """Work lists of 1024 entries or more start where the other CTAs of their head are
+    loading (a position left in the workspace by earlier CTAs and launches) and wrap
+    around. Three launches over 1032 key blocks, each against the oracle; then with
+    the deterministic switch two launches bit for bit equal."""
+    w = small_workload(3, seq_len=132096, chunk=512, hq=4, hkv=1, n_planted=8)
+    dev, cpu = layer_inputs(w)
+    ctx = make_ctx(w)
+    cs, e = w.seq_len - w.chunk, w.seq_len
+    V, S = _random_sets(np.random.default_rng(9), w.hq, e, 0.2, 0.05)
+    sets = lists_to_sets(V, S, e, e)
+    qc = dev["q"][:, cs:e].contiguous()
+    runs = []
+    for _ in range(3):
+        out, lse = ctx.sparse_prefill(qc, cs, e, dev["k"], dev["v"], sets)
+        assert ctx.status() == vsb.VS_OK
+        runs.append((f64(out), f64(lse)))
+    rows = np.arange(cs, e)
+    for h in range(w.hq):
+        oo, ol = vo.attention_rows(cpu["q"][h, cs:e], rows, cpu["k"][0], cpu["v"][0], e, vo.membership(e, V[h]),
+                                   vo.membership(e, S[h]), w.rope_base, scale_of(w), round_out=False)
+        for i, (out, lse) in enumerate(runs):
+            assert_outputs_close(out[h], oo, f"run {i} h={h}", w=w)
+            assert np.allclose(lse[h], ol, rtol=0, atol=2e-3), (i, h, np.abs(lse[h] - ol).max())
+    ctx.set_deterministic(True)
+    a = [t.clone() for t in ctx.sparse_prefill(qc, cs, e, dev["k"], dev["v"], sets)]
+    b = ctx.sparse_prefill(qc, cs, e, dev["k"], dev["v"], sets)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
 def _check_layer(name, w, keep, ref, out):
     """Per chunk and head: identical sets give outputs within tolerance; sets that
     differ under the same budgets differ only by near-ties; other budgets are only
@@ -439,14 +469,19 @@ def test_empty_and_out_of_range_sizes_are_rejected():
     assert ctx.status() == vsb.VS_OK
 
 
+@pytest.mark.parametrize("heads", [(4, 2), (40, 8)])
 @pytest.mark.parametrize("dca", [None, (2048, 256)])
-def test_sparse_prefill_gathers_scattered_verticals(dca):
+def test_sparse_prefill_gathers_scattered_verticals(dca, heads):
     """A band of slash offsets plus scattered vertical columns (before each chunk and
     inside it), the shape in which the kernel gathers vertical columns into dense
-    groups instead of executing their key blocks: every row against the oracle, and
-    the executed tiles far below the causal dense count. With DCA (stride 1792) the
-    groups are split at DCA chunk boundaries, each with its own query rotation."""
-    w = small_workload(2, seq_len=6144, chunk=2048, hq=4, hkv=2, n_planted=8)
+    groups instead of executing their key blocks: every row against the oracle (with
+    40 heads, the first and last row of every query tile and 64 random rows per chunk),
+    and the executed tiles far below the causal dense count. With DCA (stride 1792) the
+    groups are split at DCA chunk boundaries, each with its own query rotation. 40 heads
+    give 320 attention CTAs per chunk, more than two waves of one CTA per SM, so lists
+    swept from their end (every other wave) are covered too."""
+    hq, hkv = heads
+    w = small_workload(2, seq_len=6144, chunk=2048, hq=hq, hkv=hkv, n_planted=8)
     dev, cpu = layer_inputs(w)
     ctx = make_ctx(w, dca=dca)
     rng = np.random.default_rng(21)
@@ -469,14 +504,17 @@ def test_sparse_prefill_gathers_scattered_verticals(dca):
         ex, _ = ctx.prefill_stats()
         executed += ex
         dense_tiles += w.hq * sum((r0 // 128 + 1) for r0 in range(cs, e, 128))
-        got = f64(out[:, cs:e])
         rows = np.arange(cs, e)
+        if w.hq > 4:
+            tile_ends = np.concatenate([np.arange(cs, e, 128), np.minimum(np.arange(cs, e, 128) + 127, e - 1)])
+            rows = np.union1d(tile_ends, rng.choice(rows, 64, replace=False))
+        got = f64(out[:, rows])
         for h in range(w.hq):
             vh, sh = V[h][V[h] < e], S[h][S[h] < e]
-            oo, _ = vo.attention_rows(cpu["q"][h, cs:e], rows, cpu["k"][h // w.group], cpu["v"][h // w.group], e,
+            oo, _ = vo.attention_rows(cpu["q"][h, rows], rows, cpu["k"][h // w.group], cpu["v"][h // w.group], e,
                                       vo.membership(e, vh), vo.membership(e, sh), w.rope_base, scale, dca,
                                       round_out=False)
-            assert_outputs_close(got[h], oo, f"gather dca={dca} cs={cs} h={h}", w=w)
+            assert_outputs_close(got[h], oo, f"gather dca={dca} hq={w.hq} cs={cs} h={h}", w=w)
     assert executed < 0.5 * dense_tiles, (executed, dense_tiles)
 
 
