@@ -52,7 +52,8 @@ DATASHEET_BF16_TFLOPS = 2250.0
 # taken on: a sha256 prefix over attn.cu, sm100.cuh and internal.cuh. A changed
 # kernel reports null until it is captured again.
 ATTN_TRAFFIC = {
-    "cfg2_qwen7b_n32k_refine": ("d95398d87095c930", 602235136 + 201519104),
+    # one step's 32 launches averaged (the 1-pass launch list of the whole step)
+    "cfg5_14b_n1m_dca256k_refine": ("a9347671274814d5", 23130152608),
 }
 
 

@@ -96,8 +96,8 @@ VS_API vs_status vs_context_reset(vs_ctx* ctx);
 /* Wall-time limit (ns) of every bounded device wait; default 2e9. */
 VS_API vs_status vs_set_wait_limit(vs_ctx* ctx, uint64_t ns);
 /* Summation order of vs_sparse_prefill (default off). Off: a CTA whose work list has
- * 1024 entries or more starts its sweep where the other CTAs of its head are loading
- * now and wraps around, so that the CTAs in flight share each K/V block in L2 once a
+ * 1024 entries or more starts its sweep where the CTAs of its KV head are loading now
+ * and wraps around, so that the CTAs in flight share each K/V block in L2 once a
  * KV head's keys and values outgrow it; the online softmax then adds the blocks in an
  * order that depends on timing, and results may differ in the last bits from run to
  * run (each within the same rounding bounds). On: every list is swept from its start

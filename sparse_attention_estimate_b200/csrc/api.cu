@@ -90,7 +90,7 @@ Layout make_layout(const vs_attn_cfg& cfg, int64_t max_seq, int64_t max_chunk) {
   L.gkoff = take(static_cast<size_t>(hq) * (L.nkmax + 1) * sizeof(int32_t));
   L.sched = take(static_cast<size_t>(hq) * L.npairs * 2 * L.nsched * sizeof(int32_t));
   L.sched_cnt = take(static_cast<size_t>(hq) * L.npairs * sizeof(int32_t));
-  L.sweep = take(static_cast<size_t>(hq) * sizeof(int32_t));
+  L.sweep = take(static_cast<size_t>(hkv) * sizeof(int32_t));
   L.total = off;
   return L;
 }

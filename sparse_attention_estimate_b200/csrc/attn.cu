@@ -38,7 +38,7 @@ namespace vs {
 
 constexpr int kAttnThreads = 384;
 // Work lists of at least this many entries (K and V of 1024 key blocks per KV head: 64 MB)
-// are swept from where the other CTAs of their head are loading (see attn_kernel).
+// are swept from where the CTAs of their KV head are loading (see attn_kernel).
 constexpr int kSweepMin = 1024;
 // Register budgets after the role split: warpgroup 0 (TMA producer, MMA issuer, two
 // idle warps) keeps 112 per thread, the two softmax warpgroups take 192 each:
@@ -413,7 +413,7 @@ struct AttnParams {
   const int4* gtab;
   int64_t e_pad, gcap;
   int dca_sblk;  // key blocks per DCA chunk (S / 128), 0 without DCA
-  int* sweep;    // per query head: list position last loaded by one of its CTAs (a hint)
+  int* sweep;    // per KV head: list position last loaded by one of its CTAs (a hint)
   int rotate;    // lists of kSweepMin entries or more start at that position
   // row sources of the gathered groups: rotated keys and values, [hkv][rows][128]
   const uint16_t* k_rot;
@@ -509,18 +509,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     mbar_init(&s.o_final, 1);
     mbar_init(&s.drain, 1);
     s.abort_word = 0;
-    // Sweep start: where a CTA of the same query head loaded last. Once a KV head's keys
-    // and values outgrow L2, CTAs that all sweep from block 0 drift apart (SMs run at
-    // slightly different speeds, and each takes the next CTA when its own ends) until the
-    // blocks a CTA reads have left L2 before the next one reaches them. Joining the CTAs
-    // in flight keeps them within a few hundred blocks of each other. The position is kept
-    // per query head, not per KV head: heads whose masks cost different time per block
-    // then form one group each instead of one spread-out group. A list of n entries is
-    // stored twice in a row, so the sweep start .. start + n - 1 needs no wrap-around;
-    // the order of the entries changes only the summation order of the online softmax.
+    // Sweep start: where a CTA of the same KV head loaded last. Once a KV head's keys and
+    // values outgrow L2, CTAs that all sweep from block 0 drift apart (SMs run at slightly
+    // different speeds, and each takes the next CTA when its own ends) until the blocks a
+    // CTA reads have left L2 before the next one reaches them. Joining the CTAs in flight
+    // keeps them within a few hundred blocks of each other. The position is kept per KV
+    // head: all its query heads read the same blocks (one position per query head let the
+    // heads settle at different places, each group reading the blocks on its own). A list
+    // of n entries is stored twice in a row, so the sweep start .. start + n - 1 needs no
+    // wrap-around; the order of the entries changes only the summation order of the
+    // online softmax.
     int start = 0;
     if (p.rotate && n >= kSweepMin)
-      start = static_cast<int>(static_cast<uint32_t>(__ldcg(p.sweep + h)) % static_cast<uint32_t>(n));
+      start = static_cast<int>(static_cast<uint32_t>(__ldcg(p.sweep + hk)) % static_cast<uint32_t>(n));
     s.start = start;
     fence_barrier_init();
   }
@@ -581,7 +582,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
           if (p.rotate && n >= kSweepMin && (j & 63) == 0) {  // where this CTA is now
             const int pos = start + j;
-            __stcg(p.sweep + h, pos >= n ? pos - n : pos);
+            __stcg(p.sweep + hk, pos >= n ? pos - n : pos);
           }
           if (j > 0) {
             const int kc = entry_kchunk(cur, p.gtab, p.gcap, h, p.dca_sblk);

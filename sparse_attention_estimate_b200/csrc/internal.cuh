@@ -72,7 +72,7 @@ struct Layout {
   size_t gkoff;               // first group of each DCA key chunk [hq][nkmax + 1]
   size_t sched, sched_cnt;    // work lists [hq][npairs][2 * nsched] (each list written twice in a row)
                               // and their lengths [hq][npairs]
-  size_t sweep;               // list position of each query head's attention CTAs [hq] (a hint)
+  size_t sweep;               // list position of each KV head's attention CTAs [hkv] (a hint)
   size_t total;
   int64_t rows_pad;           // max_chunk rounded up to 256
   int64_t e_pad;              // max_seq rounded up to 128

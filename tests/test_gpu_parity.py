@@ -11,7 +11,7 @@ import sparse_attention_estimate_b200 as vsb
 from sparse_attention_estimate_b200 import build as vsbuild
 from tests.gpu_common import (OUT_MAX_ABS, TAU_SLACK, assert_near_tie_equal, assert_outputs_close, f64,
                               layer_inputs, lists_to_sets, make_ctx, scale_of, sets_to_lists)
-from workloads import generate_layer, small_workload
+from workloads import generate_head, generate_layer, small_workload, structure
 
 pytestmark = pytest.mark.gpu
 
@@ -311,32 +311,44 @@ def test_sparse_prefill_is_deterministic(case):
 
 
 def test_long_lists_swept_from_a_shared_start():
-    """Work lists of 1024 entries or more start where the other CTAs of their head are
-    loading (a position left in the workspace by earlier CTAs and launches) and wrap
-    around. Three launches over 1032 key blocks, each against the oracle; then with
-    the deterministic switch two launches bit for bit equal."""
-    w = small_workload(3, seq_len=132096, chunk=512, hq=4, hkv=1, n_planted=8)
-    dev, cpu = layer_inputs(w)
-    ctx = make_ctx(w)
+    """Work lists of 1024 entries or more start where the CTAs of their KV head are
+    loading and wrap around. 40 query heads over 8 KV heads, 1024 query rows (4 tile
+    pairs) against 132096 keys (1032 blocks): 160 attention CTAs, so those that start
+    after the first wave join their KV head's sweep part-way along the list. Three
+    launches, each against the oracle on the first and last row of every query tile and
+    32 random rows per head; then, with the deterministic switch, two launches bit for
+    bit equal."""
+    w = small_workload(3, seq_len=132096, chunk=1024, hq=40, hkv=8, n_planted=8)
+    st = structure(w)
     cs, e = w.seq_len - w.chunk, w.seq_len
+    q = torch.stack([generate_head(w, "q", h, rows=torch.arange(cs, e), st=st) for h in range(w.hq)])
+    k = torch.stack([generate_head(w, "k", h, st=st) for h in range(w.hkv)])
+    v = torch.stack([generate_head(w, "v", h, st=st) for h in range(w.hkv)])
+    dq, dk, dv = q.cuda(), k.cuda(), v.cuda()
+    ctx = make_ctx(w)
     V, S = _random_sets(np.random.default_rng(9), w.hq, e, 0.2, 0.05)
     sets = lists_to_sets(V, S, e, e)
-    qc = dev["q"][:, cs:e].contiguous()
     runs = []
     for _ in range(3):
-        out, lse = ctx.sparse_prefill(qc, cs, e, dev["k"], dev["v"], sets)
+        out, lse = ctx.sparse_prefill(dq, cs, e, dk, dv, sets)
         assert ctx.status() == vsb.VS_OK
         runs.append((f64(out), f64(lse)))
-    rows = np.arange(cs, e)
-    for h in range(w.hq):
-        oo, ol = vo.attention_rows(cpu["q"][h, cs:e], rows, cpu["k"][0], cpu["v"][0], e, vo.membership(e, V[h]),
-                                   vo.membership(e, S[h]), w.rope_base, scale_of(w), round_out=False)
-        for i, (out, lse) in enumerate(runs):
-            assert_outputs_close(out[h], oo, f"run {i} h={h}", w=w)
-            assert np.allclose(lse[h], ol, rtol=0, atol=2e-3), (i, h, np.abs(lse[h] - ol).max())
+    rng = np.random.default_rng(10)
+    starts = np.arange(cs, e, 128)
+    rows = np.union1d(np.concatenate([starts, starts + 127]), rng.choice(np.arange(cs, e), 32, replace=False))
+    qh, kh, vh = f64(q), f64(k), f64(v)
+    for hk in range(w.hkv):
+        kr = vo.rope(kh[hk], np.arange(e), w.rope_base)
+        for h in range(hk * w.group, (hk + 1) * w.group):
+            oo, ol = vo.attention_rows(qh[h, rows - cs], rows, kh[hk], vh[hk], e, vo.membership(e, V[h]),
+                                       vo.membership(e, S[h]), w.rope_base, scale_of(w), k_rot=kr,
+                                       round_out=False)
+            for i, (out, lse) in enumerate(runs):
+                assert_outputs_close(out[h, rows - cs], oo, f"run {i} h={h}", w=w)
+                assert np.allclose(lse[h, rows - cs], ol, rtol=0, atol=2e-3), (i, h)
     ctx.set_deterministic(True)
-    a = [t.clone() for t in ctx.sparse_prefill(qc, cs, e, dev["k"], dev["v"], sets)]
-    b = ctx.sparse_prefill(qc, cs, e, dev["k"], dev["v"], sets)
+    a = [t.clone() for t in ctx.sparse_prefill(dq, cs, e, dk, dv, sets)]
+    b = ctx.sparse_prefill(dq, cs, e, dk, dv, sets)
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
 
 
