@@ -48,12 +48,13 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # roofline denominator.
 DATASHEET_BF16_TFLOPS = 2250.0
 # DRAM bytes (read + write) of one attention-kernel launch, from one ncu capture per
-# workload (the attention-kernel summaries under profiles/), valid only for the kernel sources they were
+# workload (the launch-list summaries under profiles/), valid only for the kernel sources they were
 # taken on: a sha256 prefix over attn.cu, sm100.cuh and internal.cuh. A changed
 # kernel reports null until it is captured again.
 ATTN_TRAFFIC = {
     # one step's 32 launches averaged (the 1-pass launch list of the whole step)
     "cfg5_14b_n1m_dca256k_refine": ("a9347671274814d5", 23130152608),
+    "cfg9_14b_n1m_dca256k_refine_structured": ("a9347671274814d5", 13509399688),
 }
 
 
