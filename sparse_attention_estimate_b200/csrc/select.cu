@@ -141,9 +141,21 @@ __global__ void __launch_bounds__(kSelThreads) radix_hist_kernel(
   const int nu = st.nu;
   if (nu == 0) return;
   extern __shared__ uint32_t hist[];  // [nu][256]
-  __shared__ uint32_t up[kMaxLevels];
+  __shared__ uint32_t sp[kMaxLevels];  // the distinct prefixes, ascending
+  __shared__ int su[kMaxLevels];       // their slots in the state
   for (int i = tid; i < nu * 256; i += blockDim.x) hist[i] = 0u;
-  if (tid < nu) up[tid] = st.uprefix[tid];
+  if (tid == 0) {
+    for (int i = 0; i < nu; ++i) {  // insertion sort of at most kMaxLevels prefixes
+      const uint32_t v = st.uprefix[i];
+      int j = i;
+      for (; j > 0 && sp[j - 1] > v; --j) {
+        sp[j] = sp[j - 1];
+        su[j] = su[j - 1];
+      }
+      sp[j] = v;
+      su[j] = i;
+    }
+  }
   __syncthreads();
   const float* x = sel_row(vert, slash, e_ld, h, arr);
   const int64_t lo = static_cast<int64_t>(b) * seg, hi = min(lo + seg, e);
@@ -157,17 +169,27 @@ __global__ void __launch_bounds__(kSelThreads) radix_hist_kernel(
       uint32_t digit = 0;
       if (j0 + q < hi) {
         const uint32_t hp = shift == 24 ? 0u : (k[q] >> (shift + 8));
-        for (int uu = 0; uu < nu; ++uu)
-          if (up[uu] == hp) {
-            u = uu;
-            break;
-          }
+        int l0 = 0, l1 = nu;  // bisection: first sorted prefix >= hp
+        while (l0 < l1) {
+          const int mid = (l0 + l1) >> 1;
+          if (sp[mid] < hp)
+            l0 = mid + 1;
+          else
+            l1 = mid;
+        }
+        if (l0 < nu && sp[l0] == hp) u = su[l0];
         digit = (k[q] >> shift) & 255u;
       }
-      // equal (prefix, digit) pairs of the warp add once
-      const uint32_t tag = u < 0 ? 0xFFFFFFFFu : ((static_cast<uint32_t>(u) << 8) | digit);
-      const uint32_t peers = __match_any_sync(0xffffffffu, tag);
-      if (u >= 0 && (__ffs(peers) - 1) == (tid & 31)) atomicAdd(&hist[u * 256 + digit], __popc(peers));
+      if (shift == 24) {
+        // first digit (sign and high exponent bits): scores of one array share a few
+        // values, so equal digits of the warp add once
+        const uint32_t tag = u < 0 ? 0xFFFFFFFFu : digit;
+        const uint32_t peers = __match_any_sync(0xffffffffu, tag);
+        if (u >= 0 && (__ffs(peers) - 1) == (tid & 31)) atomicAdd(&hist[digit], __popc(peers));
+      } else if (u >= 0) {
+        // lower digits spread over the bins: a plain shared-memory add per key
+        atomicAdd(&hist[u * 256 + digit], 1u);
+      }
     }
   }
   __syncthreads();
@@ -242,10 +264,29 @@ __device__ __forceinline__ int load_thresholds(const uint32_t* thr, int h, int a
       while (u < nu && uT[u] != p[0]) ++u;
       if (u == nu) uT[nu++] = p[0];
     }
+    for (int i = 1; i < nu; ++i) {  // ascending, for the bisection of find_threshold
+      const uint32_t v = uT[i];
+      int j = i;
+      for (; j > 0 && uT[j - 1] > v; --j) uT[j] = uT[j - 1];
+      uT[j] = v;
+    }
     nu_s = nu;
   }
   __syncthreads();
   return nu_s;
+}
+
+// Index of key k among the nu distinct threshold keys uT (ascending), -1 if none.
+__device__ __forceinline__ int find_threshold(const uint32_t* uT, int nu, uint32_t k) {
+  int l0 = 0, l1 = nu;
+  while (l0 < l1) {
+    const int mid = (l0 + l1) >> 1;
+    if (uT[mid] < k)
+      l0 = mid + 1;
+    else
+      l1 = mid;
+  }
+  return (l0 < nu && uT[l0] == k) ? l0 : -1;
 }
 
 // Per segment: how many elements equal each distinct threshold key, into
@@ -266,12 +307,10 @@ __global__ void __launch_bounds__(kSelThreads) eq_count_kernel(
     load_keys4(x, j0, hi, arr, vec, k);
 #pragma unroll
     for (int q = 0; q < 4; ++q)
-      if (j0 + q < hi)
-        for (int u = 0; u < nu; ++u)
-          if (k[q] == uT[u]) {
-            atomicAdd(&c_s[u], 1);
-            break;
-          }
+      if (j0 + q < hi) {
+        const int u = find_threshold(uT, nu, k[q]);
+        if (u >= 0) atomicAdd(&c_s[u], 1);
+      }
   }
   __syncthreads();
   if (tid < kMaxLevels) cnt[(static_cast<int64_t>(h * 2 + arr) * gridDim.x + b) * kMaxLevels + tid] = c_s[tid];
@@ -303,15 +342,7 @@ __global__ void __launch_bounds__(kSelThreads) levels_kernel(
     load_keys4(x, j0, hi, arr, vec, k);
     int myu[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      myu[q] = -1;
-      if (j0 + q < hi)
-        for (int u = 0; u < nu; ++u)
-          if (k[q] == uT[u]) {
-            myu[q] = u;
-            break;
-          }
-    }
+    for (int q = 0; q < 4; ++q) myu[q] = j0 + q < hi ? find_threshold(uT, nu, k[q]) : -1;
     long long rk[4] = {0, 0, 0, 0};
     const bool mine = myu[0] >= 0 || myu[1] >= 0 || myu[2] >= 0 || myu[3] >= 0;
     if (__syncthreads_or(mine)) {
@@ -332,15 +363,29 @@ __global__ void __launch_bounds__(kSelThreads) levels_kernel(
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       uint32_t level = 255;
-      if (j0 + q < hi)
-        for (int t = 0; t < nlev; ++t) {
+      if (j0 + q < hi) {
+        // The thresholds do not increase with the level (the budgets grow), so the
+        // levels whose threshold is at most the key are a suffix: find its start t0 by
+        // bisection. Levels with no threshold (kNoThreshold) precede the others.
+        int lo_t = 0, hi_t = nlev;  // first t with T[t] <= key (T[t] != kNoThreshold)
+        while (lo_t < hi_t) {
+          const int mid = (lo_t + hi_t) >> 1;
+          const uint32_t tt = T[mid];
+          if (tt != kNoThreshold && tt <= k[q])
+            hi_t = mid;
+          else
+            lo_t = mid + 1;
+        }
+        // from t0 on: a key above the threshold is selected; a key equal to it is
+        // selected among the first take[t] equal keys (the next levels take more)
+        for (int t = lo_t; t < nlev; ++t) {
           const uint32_t tt = T[t];
-          if (tt == kNoThreshold) continue;
-          if (k[q] > tt || (k[q] == tt && rk[q] < static_cast<long long>(take[t]))) {
+          if (k[q] > tt || rk[q] < static_cast<long long>(take[t])) {
             level = static_cast<uint32_t>(t);
             break;
           }
         }
+      }
       packed |= level << (8 * q);
     }
     if (j0 + 3 < hi)
