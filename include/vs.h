@@ -187,7 +187,10 @@ VS_API vs_status vs_calibrate_accumulate(vs_ctx* ctx, const int32_t* kv_budget, 
  * h / (hq/hkv). q: [hq][q_rows][128] (row r at position q_pos0 + r, e - q_pos0
  * <= q_rows <= max_chunk); k, v: [hkv][kv_rows][128]; out: [hq][q_rows][128]
  * bf16 (rows of the chunk written, others untouched); lse_out: nullable
- * [hq][q_rows] fp32 natural-log softmax normaliser of each row.
+ * [hq][q_rows] fp32 natural-log softmax normaliser of each row. The order in
+ * which the blocks of a long work list are added follows the other CTAs in
+ * flight (see vs_set_deterministic), so results may differ in the last bits
+ * from run to run unless the context is set deterministic.
  */
 VS_API vs_status vs_sparse_prefill(vs_ctx* ctx, const uint16_t* q, int64_t q_rows, int64_t q_pos0,
                             int64_t e, const uint16_t* k, const uint16_t* v, int64_t kv_rows,

@@ -507,13 +507,13 @@ __global__ void sums_fixup_kernel(const float* __restrict__ part_v, const float*
 // recall_base_finish_kernel (the result does not depend on scheduling), which sets
 // dec[h] = 1 when the recall reaches tau: the head then needs no histogram of the
 // higher levels.
-constexpr int kBaseRound = 4096;  // columns per round of the base-recall scan
+constexpr int kBaseBatch = 4096;  // columns per batch of the base-recall scan
 __global__ void __launch_bounds__(256) recall_base_kernel(
     const float* __restrict__ vert, const float* __restrict__ slash, int64_t e_ld, int64_t e, int nr,
     const uint8_t* __restrict__ lvl, int64_t e_pad, const float* __restrict__ lse,
     const uint16_t* __restrict__ q_est, int ntile, const uint16_t* __restrict__ k_rot, int64_t k_rows, int g,
     float scale_log2, double* __restrict__ part) {
-  __shared__ int32_t queue[kBaseRound];
+  __shared__ int32_t queue[kBaseBatch];
   __shared__ int nq;
   __shared__ double red[256];
   const int h = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -534,7 +534,7 @@ __global__ void __launch_bounds__(256) recall_base_kernel(
     lse2[t] = r < nr ? lse[static_cast<int64_t>(h) * kEstRows + r] * kLog2e : 0.f;
   }
   double acc = 0.0;  // vertical + slash - both
-  for (int64_t rb = j0; rb < j1; rb += kBaseRound) {
+  for (int64_t rb = j0; rb < j1; rb += kBaseBatch) {
     if (tid == 0) nq = 0;
     __syncthreads();
     const int64_t jb = rb + 16 * tid;
@@ -582,7 +582,7 @@ __global__ void __launch_bounds__(256) recall_base_kernel(
         acc -= exp2f(dot * scale_log2 - lse2[t]);
       }
     }
-    __syncthreads();  // the queue is refilled next round
+    __syncthreads();  // the queue is refilled by the next batch
   }
   red[tid] = acc;
   __syncthreads();
