@@ -231,6 +231,26 @@ def test_recall_is_exp_of_lse_difference(rng):
     assert vo.recall(a, rows, inV, inS) == pytest.approx(np.mean(per), rel=1e-12)
 
 
+@pytest.mark.parametrize("kv,ks", [(3, 2), (7, 4), (20, 30), (40, 40)])
+def test_recall_is_vertical_plus_slash_mass_minus_their_overlap(rng, kv, ks):
+    # The mass of the selected elements is the mass of the selected columns (their
+    # vertical sums) plus that of the selected offsets (their slash sums), minus the
+    # elements both select, counted twice: the identity by which the recall at the
+    # base budgets is taken from the estimation pass's sums.
+    lse, vert, slash, a = _tiny_estimation(rng)
+    e, nr = vert.shape[0], a.shape[0]
+    rows = np.arange(e - nr, e)
+    V, S = vo.select(vert, slash, kv, ks)
+    inV, inS = vo.membership(e, V), vo.membership(e, S)
+    both = 0.0
+    for r, i in enumerate(rows):
+        for j in range(int(i) + 1):
+            if inV[j] and inS[int(i) - j]:
+                both += a[r, j]
+    mass = vert[inV].sum() + slash[inS].sum() - both
+    assert vo.recall(a, rows, inV, inS) == pytest.approx(mass / nr, rel=1e-12, abs=1e-15)
+
+
 def test_recall_full_mask_is_one_and_monotone(rng):
     lse, vert, slash, a = _tiny_estimation(rng)
     e = vert.shape[0]
